@@ -1,0 +1,408 @@
+"""Benchmark of the W4A4 quantized linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload I] [--impl kq|reference]
+
+A step is one pass of the whole online path over one batch of M tokens: per-token
+centring, block transform, MXFP4 quantization and the low-rank input (quantize kernels),
+then the block-scaled FP4 GEMM with the fused low-rank and rank-1 branches. The weights
+are prepared once, offline (reported separately as prepare_ms, not in tokens/s).
+
+Default workload: PixArt-Sigma-shaped MLP fc1 (M=4096 tokens, K=1152, N=4608, permuted
+block-Hadamard transform, rank-32 branch), bf16 output. Inputs are seeded synthetic
+data (see the ``synthetic`` package) already resident in HBM; six rotating buffer sets
+(activations, workspace, outputs and weight copies, > 2x the 126 MB L2) keep successive
+steps from hitting in L2. Steps are replayed from a CUDA graph; timing uses CUDA events on
+the launching stream, max over ranks. For N > 1 every rank runs its own batch (tokens
+are independent: weak scaling, no collective on the data path).
+
+One JSON line is printed by rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4 linear tokens/s; quantize HBM GB/s and GEMM FP4 TFLOPS as % of roofline"
+DEFAULT_WORKLOAD = 2
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16": float(p["bf16_tflops"]),
+                "bf16_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# nominal dense ratio FP4 : BF16 on B200 (9 : 2.25 PFLOP/s)
+FP4_OVER_BF16 = 4.0
+
+
+class Clocks:
+    """nvidia-smi sampler for the SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.dev}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict | None:
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sms, maxs, reasons = [], [], set()
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, mx = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            sms.append(sm)
+            maxs.append(mx)
+            names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxs),
+                "reasons": sorted(reasons), "samples": len(sms)}
+
+
+def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = None):
+    """Time the CPU oracle's online path (centre, transform, encode, fp64 contraction with
+    both branches) on the first rows of the batch for about budget_s seconds."""
+    from oracle import layer as olayer
+    X = inp["X"]
+    olayer.linear(X[:8], inp["T"], w.center, prep)            # warm caches
+    t0 = time.perf_counter()
+    olayer.linear(X[:32], inp["T"], w.center, prep)
+    per_row = max((time.perf_counter() - t0) / 32, 1e-6)
+    rows = int(min(max_rows or w.M, max(32, budget_s / per_row)))
+    t0 = time.perf_counter()
+    done = 0
+    while done < rows:
+        n = min(512, rows - done)
+        olayer.linear(X[done:done + n], inp["T"], w.center, prep)
+        done += n
+    dt = time.perf_counter() - t0
+    return done / dt, done, dt
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def run_reference(args, w):
+    """The oracle on the host cores, same workload/metric/unit (bounded sample per step)."""
+    from oracle import layer as olayer
+    from synthetic import make_inputs
+    inp = make_inputs(w)
+    prep = olayer.prepare(inp["W"], inp["T"], w.rank)
+    X = inp["X"]
+    t0 = time.perf_counter()
+    olayer.linear(X[:32], inp["T"], w.center, prep)
+    per_row = max((time.perf_counter() - t0) / 32, 1e-6)
+    total_steps = max(1, args.steps + args.warmup)
+    rows = int(np.clip(120.0 / total_steps / per_row, 1, w.M))
+    for i in range(args.warmup):
+        olayer.linear(X[:rows], inp["T"], w.center, prep)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        olayer.linear(X[:rows], inp["T"], w.center, prep)
+    dt = time.perf_counter() - t0
+    value = rows * args.steps / dt
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.label, "tokens_per_step": rows, "global_batch": w.M},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"first {rows} of {w.M} tokens per step, {args.steps} steps"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50000)
+    ap.add_argument("--warmup", type=int, default=30)
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", choices=["kq", "reference"], default="kq")
+    ap.add_argument("--out", choices=["bf16", "f32"], default="bf16")
+    ap.add_argument("--sets", type=int, default=0, help="rotating buffer sets (0 = auto)")
+    ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    from synthetic import workload
+    w = workload(args.workload)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    import w4a4_post_quantization_token_b200 as kq
+    from synthetic import make_inputs
+
+    inp = make_inputs(w)
+    L = kq.Layer(w.K, w.N, w.rank, w.center, inp["T"])
+    out_bf16 = args.out == "bf16"
+    ydt = torch.bfloat16 if out_bf16 else torch.float32
+    odt = kq.OUT_BF16 if out_bf16 else kq.OUT_F32
+
+    # offline preparation on the GPU (timed separately)
+    W = inp["W"].to(dev)
+    wbuf0 = torch.empty(kq.weights_bytes(L), dtype=torch.uint8, device=dev)
+    ws = torch.empty(kq.prepare_ws_bytes(L), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    kq.prepare_weights(L, W, wbuf0, ws)
+    torch.cuda.synchronize()
+    prepare_ms = (time.perf_counter() - t0) * 1e3
+    del ws, W
+
+    # rotating buffer sets
+    X0 = inp["X"].to(dev)
+    abytes = kq.act_bytes(L, w.M)
+    set_bytes = X0.numel() * 2 + abytes + w.M * w.N * (2 if out_bf16 else 4) + wbuf0.numel()
+    R = args.sets or max(2, int(np.ceil(2 * 126e6 / set_bytes)) + 1)
+    sets = []
+    for j in range(R):
+        Xj = X0 if j == 0 else X0.clone()
+        wj = wbuf0 if j == 0 else wbuf0.clone()
+        sets.append({"X": Xj, "w": wj,
+                     "act": torch.empty(abytes, dtype=torch.uint8, device=dev),
+                     "Y": torch.empty((w.M, w.N), dtype=ydt, device=dev)})
+    stream = torch.cuda.current_stream()
+
+    def step(j, ev=None):
+        s = sets[j]
+        cur = torch.cuda.current_stream()
+        if ev is not None:
+            ev[0].record(cur)
+        kq.quantize_act(L, s["w"], s["X"], s["act"])
+        if ev is not None:
+            ev[1].record(cur)
+        kq.gemm(L, s["w"], s["act"], w.M, s["Y"], odt)
+        if ev is not None:
+            ev[2].record(cur)
+
+    for i in range(args.warmup):
+        step(i % R)
+    torch.cuda.synchronize()
+    for s in sets:
+        assert kq.last_device_error(L, s["act"], w.M) == 0
+
+    # CUDA graph of one rotation (R steps) with per-phase events
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(R)]
+    graph = None
+    if not args.no_graph:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, capture_error_mode="relaxed"):
+                for j in range(R):
+                    step(j, evs[j])
+            graph.replay()
+            torch.cuda.synchronize()
+        except Exception as e:  # pragma: no cover - fall back to eager launches
+            print(f"# graph capture failed ({e}); timing eager launches", file=sys.stderr)
+            graph = None
+            stream = torch.cuda.current_stream()
+
+    clocks = Clocks(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    if graph is not None:
+        full, rem = divmod(args.steps, R)
+        for _ in range(full):
+            graph.replay()
+        for j in range(rem):
+            step(j)
+        # per-phase event times come from the last complete replay
+        if full == 0:
+            graph.replay()
+    else:
+        for i in range(args.steps):
+            step(i % R, evs[i % R])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        dist.barrier()
+
+    q_ms = float(np.mean([evs[j][0].elapsed_time(evs[j][1]) for j in range(R)]))
+    g_ms = float(np.mean([evs[j][1].elapsed_time(evs[j][2]) for j in range(R)]))
+    for s in sets:
+        assert kq.last_device_error(L, s["act"], w.M) == 0
+
+    ms_per_step = elapsed_ms / args.steps
+    tokens_per_s = w.M * world * args.steps / (elapsed_ms / 1e3)
+
+    # roofline of the dominant kernel (algorithmic work per launch / event-timed duration)
+    peaks = _peaks()
+    M, K, N, rp = w.M, w.K, w.N, (64 if w.rank else 0)
+    gemm_flops = 2.0 * M * N * K + 2.0 * M * N * w.rank + (M * N if w.center else 0)
+    ybytes = M * N * (2 if out_bf16 else 4)
+    gemm_bytes = M * K / 2 + N * K / 2 + (M + N) * K / 32 + M * rp * 2 + N * rp * 2 + N * 4 + \
+        (M * 4 if w.center else 0) + ybytes
+    q_bytes = M * K * 2 + M * K / 2 + M * K / 32 + M * 4 + M * rp * 2
+    fp4_peak = peaks["bf16_sustained"] * FP4_OVER_BF16
+    t_tensor = gemm_flops / (fp4_peak * 1e12)
+    t_hbm = gemm_bytes / (peaks["hbm_gbs"] * 1e9)
+    if g_ms >= q_ms:
+        if t_tensor >= t_hbm:
+            ach = gemm_flops / (g_ms * 1e-3) / 1e12
+            roof = {"kernel": "k_gemm_mxf4", "bound": "tensor", "achieved": ach, "peak": fp4_peak,
+                    "unit": "TFLOP/s", "frac": ach / fp4_peak}
+        else:
+            ach = gemm_bytes / (g_ms * 1e-3) / 1e9
+            roof = {"kernel": "k_gemm_mxf4", "bound": "hbm", "achieved": ach,
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    else:
+        ach = q_bytes / (q_ms * 1e-3) / 1e9
+        roof = {"kernel": "k_quantize_rows+k_lowrank_u", "bound": "hbm", "achieved": ach,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    roof["traffic"] = None
+    roof["peak_source"] = peaks["source"] + (" (FP4 = 4 x sustained bf16)" if roof["unit"] == "TFLOP/s" else "")
+
+    # end-to-end through the host-buffer entry point (pinned memory, copies timed)
+    e2e = None
+    if args.e2e_steps > 0:
+        Xh = inp["X"].pin_memory()
+        Yh = torch.empty((w.M, w.N), dtype=ydt).pin_memory()
+        s0 = sets[0]
+        for _ in range(2):
+            kq.linear_host(L, s0["w"], Xh, s0["X"], Yh, s0["Y"], s0["act"], odt)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        e0.record()
+        for _ in range(args.e2e_steps):
+            kq.linear_host(L, s0["w"], Xh, s0["X"], Yh, s0["Y"], s0["act"], odt)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        e2e = {"value": w.M * world * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(w.M * w.K * 2),
+               "d2h_bytes_per_step": int(w.M * w.N * (2 if out_bf16 else 4)),
+               "steps": args.e2e_steps, "api": "kq_linear_host"}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import layer as olayer
+        prep = olayer.prepare(inp["W"], inp["T"], w.rank)
+        v, rows, dt = oracle_tokens_per_s(w, inp, prep, budget_s=12.0)
+        cpu = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
+               "sample": f"first {rows} of {w.M} tokens ({dt:.1f} s, fp64 NumPy, weights "
+                         f"prepared beforehand)"}
+
+    launches_per_step = 2 + (1 if w.rank else 0)
+    line = {
+        "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4",
+        "data": "synthetic",
+        "config": {"workload": w.label, "global_batch": w.M * world, "tokens_per_gpu": w.M,
+                   "K": K, "N": N, "transform": w.transform, "center": w.center, "rank": w.rank,
+                   "out_dtype": args.out, "parallelism": f"replicas x{world} (token-sharded)",
+                   "l2": f"{R} rotating buffer sets of {set_bytes / 1e6:.0f} MB (> L2)",
+                   "graph": graph is not None},
+        "phases_ms": {"quantize": q_ms, "gemm": g_ms},
+        "quantize_gbs": q_bytes / (q_ms * 1e-3) / 1e9,
+        "gemm_tflops": gemm_flops / (g_ms * 1e-3) / 1e12,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+        "prepare_ms": prepare_ms,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del graph
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,97 @@
+"""The C-ABI library loads and exports every symbol include/kq.h declares; host-side
+size queries and argument validation work without a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import w4a4_post_quantization_token_b200 as kq
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "kq.h")
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(kq.lib, n), f"libkq.so does not export {n}"
+    assert sorted(kq.SYMBOLS) == names
+
+
+def test_library_is_in_tree_and_versioned():
+    assert os.path.dirname(kq.library_path) == os.path.dirname(kq.__file__)
+    assert b"sm_100a" in kq.lib.kq_version()
+
+
+def test_struct_layout_matches_c():
+    # kq_transform_desc: int32 + ptr + int32 + ptr + int32 + ptr + ptr (with padding) = 56
+    assert ctypes.sizeof(kq._TransformDesc) == 56
+    assert ctypes.sizeof(kq._LayerDesc) == 16 + 56
+
+
+def _kron():
+    return {"kind": "kron", "A": np.eye(4, dtype=np.float32), "B": np.eye(8, dtype=np.float32)}
+
+
+def test_size_queries():
+    L = kq.Layer(1152, 4608, 32, False, {"kind": "rpbh", "perm": np.arange(1152),
+                                          "sign": np.ones(1152, np.int8)})
+    wb = kq.weights_bytes(L)
+    # at least codes + scales + L2^T + L1'^T + sums
+    assert wb >= 4608 * 576 + 4608 * 36 + 4608 * 64 * 2 + 144 * 1152 * 2
+    ab = kq.act_bytes(L, 4096)
+    assert ab >= 4096 * 576 + 4096 * 36 + 4096 * 64 * 2
+    assert kq.act_bytes(L, 4097) > ab
+    assert kq.act_bytes(L, 0) == 0
+
+
+@pytest.mark.parametrize("K,N,rank,status", [(1000, 64, 0, 2), (64, 40, 0, 2), (64, 64, 65, 2),
+                                              (0, 64, 0, 1), (64, 64, -1, 1)])
+def test_invalid_shapes_rejected(K, N, rank, status):
+    L = kq.Layer(K, N, rank, False, {"kind": "none"})
+    assert kq.weights_bytes(L) == 0
+    r = kq.lib.kq_quantize_act(L.desc, None, None, 4, None, 0, None)
+    assert r == status
+
+
+def test_invalid_transform_rejected():
+    K = 64
+    bad_perm = {"kind": "rpbh", "perm": np.zeros(K, np.int32), "sign": np.ones(K, np.int8)}
+    assert kq.weights_bytes(kq.Layer(K, 64, 0, False, bad_perm)) == 0
+    bad_sign = {"kind": "rpbh", "perm": np.arange(K), "sign": np.zeros(K, np.int8)}
+    assert kq.weights_bytes(kq.Layer(K, 64, 0, False, bad_sign)) == 0
+    bad_dim = {"kind": "kron", "A": np.eye(2, dtype=np.float32), "B": np.eye(16, dtype=np.float32)}
+    assert kq.weights_bytes(kq.Layer(K, 64, 0, False, bad_dim)) == 0
+    nan = {"kind": "kron", "A": np.full((4, 4), np.nan, np.float32), "B": np.eye(8, dtype=np.float32)}
+    assert kq.weights_bytes(kq.Layer(K, 64, 0, False, nan)) == 0
+    assert kq.weights_bytes(kq.Layer(K, 64, 0, False, _kron())) > 0
+
+
+def test_null_and_alignment_errors_before_any_launch():
+    L = kq.Layer(64, 64, 0, False, _kron())
+    M = 8
+    # null pointers -> invalid argument
+    assert kq.lib.kq_linear(L.desc, None, None, M, None, 0, None, 0, None) == 1
+    # misaligned device pointers -> alignment error (checked before any CUDA call)
+    odd = ctypes.c_void_p(0x1000 + 8)
+    ok = ctypes.c_void_p(0x100000)
+    assert kq.lib.kq_quantize_act(L.desc, ok, odd, M, ok, 1 << 20, None) == 3
+    # too-small workspace
+    assert kq.lib.kq_quantize_act(L.desc, ok, ok, M, ok, 16, None) == 5
+    # bad output dtype
+    assert kq.lib.kq_gemm(L.desc, ok, ok, M, ok, 7, None) == 1
+    assert kq.lib.kq_debug_encode_f32(ok, M, 33, ok, ok, None) == 2
+
+
+def test_status_strings():
+    for s in range(9):
+        assert kq.status_string(s)
+    assert "timed out" in kq.status_string(7)

@@ -1,0 +1,536 @@
+// C-ABI entry points of libkq (declared in include/kq.h): argument validation on the
+// host, TMA descriptor creation, and kernel launches on the caller's stream.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/kq.h"
+#include "kq_internal.cuh"
+#include "kq_pack.cuh"
+#include "kq_prepare.cuh"
+
+using namespace kq;
+
+namespace {
+
+// ------------------------------------------------------------------ device checks --
+struct DeviceInfo { bool ok = false; int sms = 0; };
+
+kq_status current_device(DeviceInfo* out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return KQ_ERR_CUDA;
+  static std::mutex mu;
+  static std::vector<DeviceInfo> cache;
+  std::lock_guard<std::mutex> g(mu);
+  if (static_cast<int>(cache.size()) <= dev) cache.resize(dev + 1);
+  if (!cache[dev].ok) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return KQ_ERR_CUDA;
+    if (major != 10 || minor != 0) return KQ_ERR_NO_SM100;
+    cache[dev].ok = true;
+    cache[dev].sms = sms;
+  }
+  *out = cache[dev];
+  return KQ_OK;
+}
+
+// -------------------------------------------------------------- tensor maps (TMA) --
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool encode_fn() {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  return g_encode != nullptr;
+}
+
+// 2-D tiled map: inner extent (elements), outer extent (rows), row pitch (bytes).
+bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t pitch, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle sw) {
+  if (!encode_fn()) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {pitch};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- validation --------
+bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+
+kq_status check_desc(const kq_layer_desc* d) {
+  if (!d) return KQ_ERR_INVALID_ARG;
+  if (d->K <= 0 || d->N <= 0 || d->rank < 0) return KQ_ERR_INVALID_ARG;
+  if (d->K % 32 != 0 || d->N % 16 != 0 || d->rank > kRankPad) return KQ_ERR_UNSUPPORTED_SHAPE;
+  if (d->center != 0 && d->center != 1) return KQ_ERR_INVALID_ARG;
+  switch (d->t.kind) {
+    case KQ_T_NONE: break;
+    case KQ_T_KRON:
+      if (!d->t.A || !d->t.B) return KQ_ERR_INVALID_ARG;
+      if (d->t.a_dim != 4 || d->t.b_dim != 8) return KQ_ERR_UNSUPPORTED_SHAPE;
+      for (int i = 0; i < 16; ++i) if (!std::isfinite(d->t.A[i])) return KQ_ERR_INVALID_ARG;
+      for (int i = 0; i < 64; ++i) if (!std::isfinite(d->t.B[i])) return KQ_ERR_INVALID_ARG;
+      break;
+    case KQ_T_RPBH: {
+      if (!d->t.perm || !d->t.sign) return KQ_ERR_INVALID_ARG;
+      std::vector<char> seen(static_cast<size_t>(d->K), 0);
+      for (int k = 0; k < d->K; ++k) {
+        const int32_t p = d->t.perm[k];
+        if (p < 0 || p >= d->K || seen[p]) return KQ_ERR_INVALID_ARG;
+        seen[p] = 1;
+        if (d->t.sign[k] != 1 && d->t.sign[k] != -1) return KQ_ERR_INVALID_ARG;
+      }
+      break;
+    }
+    default: return KQ_ERR_INVALID_ARG;
+  }
+  return KQ_OK;
+}
+
+WeightsLayout wlayout(const kq_layer_desc* d) {
+  return WeightsLayout::make(d->K, d->N, d->rank, d->center != 0, d->t.kind);
+}
+ActLayout alayout(const kq_layer_desc* d, int M) { return ActLayout::make(M, d->K, d->rank); }
+
+// Gauss-Jordan inverse with partial pivoting (float64); false if singular.
+bool invert(const double* a, int n, double* inv) {
+  std::vector<double> m(static_cast<size_t>(n) * 2 * n, 0.0);
+  for (int i = 0; i < n; ++i) {
+    for (int j = 0; j < n; ++j) m[i * 2 * n + j] = a[i * n + j];
+    m[i * 2 * n + n + i] = 1.0;
+  }
+  double scale = 0.0;
+  for (int i = 0; i < n * n; ++i) scale = std::fmax(scale, std::fabs(a[i]));
+  if (scale == 0.0) return false;
+  for (int c = 0; c < n; ++c) {
+    int piv = c;
+    for (int r = c + 1; r < n; ++r)
+      if (std::fabs(m[r * 2 * n + c]) > std::fabs(m[piv * 2 * n + c])) piv = r;
+    if (std::fabs(m[piv * 2 * n + c]) <= 1e-12 * scale) return false;
+    if (piv != c)
+      for (int j = 0; j < 2 * n; ++j) std::swap(m[c * 2 * n + j], m[piv * 2 * n + j]);
+    const double p = m[c * 2 * n + c];
+    for (int j = 0; j < 2 * n; ++j) m[c * 2 * n + j] /= p;
+    for (int r = 0; r < n; ++r) {
+      if (r == c) continue;
+      const double f = m[r * 2 * n + c];
+      if (f != 0.0)
+        for (int j = 0; j < 2 * n; ++j) m[r * 2 * n + j] -= f * m[c * 2 * n + j];
+    }
+  }
+  for (int i = 0; i < n; ++i)
+    for (int j = 0; j < n; ++j) inv[i * n + j] = m[i * 2 * n + n + j];
+  return true;
+}
+
+// 32x32 Kronecker block (row-major): (A (x) B)[8i + j][8k + l] = A[i][k] B[j][l]
+void kron32(const double* A, const double* B, double* P) {
+  for (int i = 0; i < 4; ++i)
+    for (int j = 0; j < 8; ++j)
+      for (int k = 0; k < 4; ++k)
+        for (int l = 0; l < 8; ++l) P[(8 * i + j) * 32 + 8 * k + l] = A[4 * i + k] * B[8 * j + l];
+}
+
+// RPBH tables as stored in the weights buffer: int32 perm, float sign/sqrt(32)
+void rpbh_tables(const kq_layer_desc* d, std::vector<float>* sgn) {
+  sgn->resize(static_cast<size_t>(d->K));
+  const float rs = static_cast<float>(1.0 / std::sqrt(32.0));
+  for (int k = 0; k < d->K; ++k) (*sgn)[k] = d->t.sign[k] < 0 ? -rs : rs;
+}
+
+kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const void* X, int M,
+                            uint8_t* act, QuantParams* p, const DeviceInfo& di) {
+  std::memset(p, 0, sizeof(*p));
+  const WeightsLayout WL = wlayout(d);
+  const ActLayout AL = alayout(d, M);
+  const int K = d->K, nb = K / kBlock;
+  int box_lines = 1;
+  for (int c = 1; c <= 256 && c <= nb; ++c) if (nb % c == 0) box_lines = c;
+  if (!make_tmap(&p->tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, 32,
+                 static_cast<uint64_t>(M) * nb, 64, 32, static_cast<uint32_t>(box_lines),
+                 CU_TENSOR_MAP_SWIZZLE_64B))
+    return KQ_ERR_CUDA;
+  if (d->t.kind == KQ_T_KRON) {
+    for (int i = 0; i < 16; ++i) p->A[i] = d->t.A[i];
+    for (int i = 0; i < 64; ++i) p->B[i] = d->t.B[i];
+  }
+  p->M = M; p->K = K; p->m_pad = static_cast<int>(AL.m_pad);
+  p->kind = d->t.kind; p->center = d->center;
+  p->katoms = sf_katoms(K);
+  p->box_lines = box_lines;
+  const size_t slot = align_up(static_cast<size_t>(K) * 2, 1024);
+  const size_t budget = 200 * 1024;
+  int nw = 8, slots = 2;
+  while (nw * slots * slot > budget && slots > 1) --slots;
+  while (nw * slots * slot > budget && nw > 1) nw >>= 1;
+  if (nw * slots * slot > budget) return KQ_ERR_UNSUPPORTED_SHAPE;
+  p->warps_per_cta = nw;
+  p->slots = slots;
+  const size_t smem = 1024 + static_cast<size_t>(nw) * slots * slot;
+  int per_sm = static_cast<int>((227 * 1024) / (smem + 1024));
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm * nw > 32) per_sm = 32 / nw > 0 ? 32 / nw : 1;   // at most 32 warps per SM
+  p->ctas_per_sm = per_sm;
+  (void)di;
+  if (act) {
+    p->codes = act + AL.codes;
+    p->sf = act + AL.sf;
+    p->mu = reinterpret_cast<float*>(act + AL.mu);
+    p->err = reinterpret_cast<uint32_t*>(act + AL.err);
+  }
+  p->perm = reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(weights) + WL.perm);
+  p->sgn = reinterpret_cast<const float*>(static_cast<const uint8_t*>(weights) + WL.sgn);
+  return KQ_OK;
+}
+
+kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* X, int M,
+                       uint8_t* act, cudaStream_t st, const DeviceInfo& di) {
+  const WeightsLayout WL = wlayout(d);
+  const ActLayout AL = alayout(d, M);
+  QuantParams qp;
+  kq_status s = fill_quant_params(d, weights, X, M, act, &qp, di);
+  if (s != KQ_OK) return s;
+  if (launch_quantize_rows(qp, false, di.sms, st) != cudaSuccess) return KQ_ERR_CUDA;
+  if (d->rank > 0) {
+    LowRankParams lp;
+    std::memset(&lp, 0, sizeof(lp));
+    if (!make_tmap(&lp.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(d->K),
+                   static_cast<uint64_t>(M), static_cast<uint64_t>(d->K) * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return KQ_ERR_CUDA;
+    if (!make_tmap(&lp.tmap_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   static_cast<const uint8_t*>(weights) + WL.l1t, static_cast<uint64_t>(d->K),
+                   kUCols, static_cast<uint64_t>(d->K) * 2, 64, kUCols, CU_TENSOR_MAP_SWIZZLE_128B))
+      return KQ_ERR_CUDA;
+    lp.c1 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(weights) + WL.c1);
+    lp.u = reinterpret_cast<uint16_t*>(act + AL.u);
+    lp.M = M; lp.K = d->K; lp.center = d->center;
+    lp.err = reinterpret_cast<uint32_t*>(act + AL.err);
+    if (launch_lowrank_u(lp, st) != cudaSuccess) return KQ_ERR_CUDA;
+  }
+  return KQ_OK;
+}
+
+kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* act, int M, void* Y,
+                   int out_dtype, cudaStream_t st) {
+  const WeightsLayout WL = wlayout(d);
+  const ActLayout AL = alayout(d, M);
+  const uint8_t* w = static_cast<const uint8_t*>(weights);
+  const int K = d->K, N = d->N;
+  const int bn = (N % 256 == 0) ? 256 : (N % 128 == 0 ? 128 : 256);
+  GemmParams gp;
+  std::memset(&gp, 0, sizeof(gp));
+  if (!make_tmap(&gp.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, act + AL.codes, static_cast<uint64_t>(K / 2),
+                 static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), 128, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return KQ_ERR_CUDA;
+  if (!make_tmap(&gp.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w + WL.rcodes, static_cast<uint64_t>(K / 2),
+                 static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), 128,
+                 static_cast<uint32_t>(bn), CU_TENSOR_MAP_SWIZZLE_128B))
+    return KQ_ERR_CUDA;
+  if (d->rank > 0) {
+    if (!make_tmap(&gp.tmap_u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act + AL.u, kRankPad,
+                   static_cast<uint64_t>(M), kRankPad * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+      return KQ_ERR_CUDA;
+    if (!make_tmap(&gp.tmap_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w + WL.l2t, kRankPad,
+                   static_cast<uint64_t>(N), kRankPad * 2, 64, static_cast<uint32_t>(bn),
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return KQ_ERR_CUDA;
+  }
+  gp.sfa = act + AL.sf;
+  gp.sfb = w + WL.rsf;
+  gp.mu = d->center ? reinterpret_cast<const float*>(act + AL.mu) : nullptr;
+  gp.s = reinterpret_cast<const float*>(w + WL.s);
+  gp.y = Y;
+  gp.M = M; gp.N = N; gp.K = K;
+  gp.rank_pad = d->rank > 0 ? kRankPad : 0;
+  gp.katoms = sf_katoms(K);
+  gp.err = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(act) + AL.err);
+  if (launch_gemm(gp, bn, out_dtype == KQ_OUT_BF16, st) != cudaSuccess) return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
+}  // namespace
+
+// =====================================================================================
+extern "C" {
+
+const char* kq_status_string(kq_status s) {
+  switch (s) {
+    case KQ_OK: return "ok";
+    case KQ_ERR_INVALID_ARG: return "invalid argument";
+    case KQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case KQ_ERR_ALIGNMENT: return "device pointer not 256-byte aligned";
+    case KQ_ERR_SINGULAR_TRANSFORM: return "Kronecker factor is singular";
+    case KQ_ERR_WORKSPACE_TOO_SMALL: return "buffer smaller than the size query";
+    case KQ_ERR_CUDA: return "CUDA call failed";
+    case KQ_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case KQ_ERR_NO_SM100: return "device is not sm_100 (B200)";
+  }
+  return "unknown status";
+}
+
+const char* kq_version(void) { return "kq 0.1 (sm_100a, tcgen05 mxf4)"; }
+
+size_t kq_weights_bytes(const kq_layer_desc* desc) {
+  if (check_desc(desc) != KQ_OK) return 0;
+  return wlayout(desc).total;
+}
+
+size_t kq_act_bytes(const kq_layer_desc* desc, int32_t M) {
+  if (check_desc(desc) != KQ_OK || M <= 0) return 0;
+  return alayout(desc, M).total;
+}
+
+size_t kq_prepare_ws_bytes(const kq_layer_desc* desc) {
+  if (check_desc(desc) != KQ_OK) return 0;
+  const size_t lw = prepare_syevd_lwork(desc->K, desc->N, desc->rank);
+  if (lw == 0) return 0;
+  return PrepareWs::make(desc->K, desc->N, desc->rank, lw).total;
+}
+
+kq_status kq_prepare_weights(const kq_layer_desc* desc, const void* W_bf16, void* weights, void* ws,
+                             size_t ws_bytes, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (!W_bf16 || !weights || !ws) return KQ_ERR_INVALID_ARG;
+  if (!aligned(W_bf16) || !aligned(weights) || !aligned(ws)) return KQ_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  const size_t lw = prepare_syevd_lwork(desc->K, desc->N, desc->rank);
+  if (lw == 0) return KQ_ERR_CUDA;
+  if (ws_bytes < PrepareWs::make(desc->K, desc->N, desc->rank, lw).total)
+    return KQ_ERR_WORKSPACE_TOO_SMALL;
+
+  double pinv[32 * 32], pfwd[32 * 32];
+  for (int i = 0; i < 32 * 32; ++i) pinv[i] = pfwd[i] = (i / 32 == i % 32) ? 1.0 : 0.0;
+  if (desc->t.kind == KQ_T_KRON) {
+    double A[16], B[64], Ai[16], Bi[64];
+    for (int i = 0; i < 16; ++i) A[i] = desc->t.A[i];
+    for (int i = 0; i < 64; ++i) B[i] = desc->t.B[i];
+    if (!invert(A, 4, Ai) || !invert(B, 8, Bi)) return KQ_ERR_SINGULAR_TRANSFORM;
+    kron32(Ai, Bi, pinv);
+    kron32(A, B, pfwd);
+  }
+  std::vector<float> sgn;
+  if (desc->t.kind == KQ_T_RPBH) rpbh_tables(desc, &sgn);
+
+  PrepareArgs a;
+  a.K = desc->K; a.N = desc->N; a.rank = desc->rank; a.kind = desc->t.kind;
+  a.center = desc->center != 0;
+  a.W = W_bf16; a.weights = weights; a.ws = ws; a.syevd_lwork = lw;
+  a.pinv_host = pinv; a.pfwd_host = pfwd;
+  a.perm_host = desc->t.kind == KQ_T_RPBH ? desc->t.perm : nullptr;
+  a.sgn_host = desc->t.kind == KQ_T_RPBH ? sgn.data() : nullptr;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  switch (run_prepare(a)) {
+    case PrepStatus::Ok: return KQ_OK;
+    case PrepStatus::Solver: return KQ_ERR_CUDA;
+    default: return KQ_ERR_CUDA;
+  }
+}
+
+kq_status kq_quantize_act(const kq_layer_desc* desc, const void* weights, const void* X_bf16,
+                          int32_t M, void* act, size_t act_bytes, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (M <= 0 || !weights || !X_bf16 || !act) return KQ_ERR_INVALID_ARG;
+  if (!aligned(weights) || !aligned(X_bf16) || !aligned(act)) return KQ_ERR_ALIGNMENT;
+  if (act_bytes < alayout(desc, M).total) return KQ_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(act, 0, 4, st) != cudaSuccess) return KQ_ERR_CUDA;
+  return run_quantize(desc, weights, X_bf16, M, static_cast<uint8_t*>(act), st, di);
+}
+
+kq_status kq_gemm(const kq_layer_desc* desc, const void* weights, const void* act, int32_t M,
+                  void* Y, int32_t out_dtype, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (M <= 0 || !weights || !act || !Y) return KQ_ERR_INVALID_ARG;
+  if (out_dtype != KQ_OUT_F32 && out_dtype != KQ_OUT_BF16) return KQ_ERR_INVALID_ARG;
+  if (!aligned(weights) || !aligned(act) || !aligned(Y)) return KQ_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  return run_gemm(desc, weights, static_cast<const uint8_t*>(act), M, Y, out_dtype,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+kq_status kq_linear(const kq_layer_desc* desc, const void* weights, const void* X_bf16, int32_t M,
+                    void* Y, int32_t out_dtype, void* act, size_t act_bytes, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (!Y) return KQ_ERR_INVALID_ARG;
+  if (out_dtype != KQ_OUT_F32 && out_dtype != KQ_OUT_BF16) return KQ_ERR_INVALID_ARG;
+  if (!aligned(Y)) return KQ_ERR_ALIGNMENT;
+  s = kq_quantize_act(desc, weights, X_bf16, M, act, act_bytes, stream);
+  if (s != KQ_OK) return s;
+  return run_gemm(desc, weights, static_cast<const uint8_t*>(act), M, Y, out_dtype,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+kq_status kq_linear_host(const kq_layer_desc* desc, const void* weights, const void* X_host,
+                         void* X_dev, int32_t M, void* Y_host, void* Y_dev, int32_t out_dtype,
+                         void* act, size_t act_bytes, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (!X_host || !Y_host || !X_dev || !Y_dev || M <= 0) return KQ_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(M) * desc->K * 2;
+  const size_t yb = static_cast<size_t>(M) * desc->N * (out_dtype == KQ_OUT_BF16 ? 2 : 4);
+  if (cudaMemcpyAsync(X_dev, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  s = kq_linear(desc, weights, X_dev, M, Y_dev, out_dtype, act, act_bytes, stream);
+  if (s != KQ_OK) return s;
+  if (cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
+kq_status kq_weights_pack(const kq_layer_desc* desc, const void* r_codes, const void* r_scales,
+                          const float* L1p_f32, const void* L2_bf16, const float* s_col,
+                          void* weights, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (!r_codes || !r_scales || !s_col || !weights) return KQ_ERR_INVALID_ARG;
+  if (desc->rank > 0 && (!L1p_f32 || !L2_bf16)) return KQ_ERR_INVALID_ARG;
+  if (!aligned(weights)) return KQ_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  const WeightsLayout WL = wlayout(desc);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(weights);
+  if (pack_weights(WL, static_cast<const uint8_t*>(r_codes), static_cast<const uint8_t*>(r_scales),
+                   L1p_f32, static_cast<const uint16_t*>(L2_bf16), s_col, w, st) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  if (desc->t.kind == KQ_T_RPBH) {
+    std::vector<float> sgn;
+    rpbh_tables(desc, &sgn);
+    if (cudaMemcpyAsync(w + WL.perm, desc->t.perm, static_cast<size_t>(desc->K) * 4,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(w + WL.sgn, sgn.data(), static_cast<size_t>(desc->K) * 4,
+                        cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return KQ_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KQ_ERR_CUDA;   // sgn is a local
+  }
+  return KQ_OK;
+}
+
+kq_status kq_weights_unpack(const kq_layer_desc* desc, const void* weights, void* r_codes,
+                            void* r_scales, float* L1p_f32, void* L2_bf16, float* c1, float* s_col,
+                            kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (!weights) return KQ_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  if (unpack_weights(wlayout(desc), static_cast<const uint8_t*>(weights),
+                     static_cast<uint8_t*>(r_codes), static_cast<uint8_t*>(r_scales), L1p_f32,
+                     static_cast<uint16_t*>(L2_bf16), c1, s_col,
+                     reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
+kq_status kq_act_pack(const kq_layer_desc* desc, const void* codes, const void* scales,
+                      const float* mu, const void* U_bf16, int32_t M, void* act, size_t act_bytes,
+                      kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (M <= 0 || !codes || !scales || !act) return KQ_ERR_INVALID_ARG;
+  if (desc->center && !mu) return KQ_ERR_INVALID_ARG;
+  if (desc->rank > 0 && !U_bf16) return KQ_ERR_INVALID_ARG;
+  if (!aligned(act)) return KQ_ERR_ALIGNMENT;
+  if (act_bytes < alayout(desc, M).total) return KQ_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  if (pack_act(alayout(desc, M), desc->rank, static_cast<const uint8_t*>(codes),
+               static_cast<const uint8_t*>(scales), mu, static_cast<const uint16_t*>(U_bf16),
+               static_cast<uint8_t*>(act), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
+kq_status kq_act_unpack(const kq_layer_desc* desc, const void* act, int32_t M, void* codes,
+                        void* scales, float* mu, void* U_bf16, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (M <= 0 || !act) return KQ_ERR_INVALID_ARG;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  if (unpack_act(alayout(desc, M), desc->rank, static_cast<const uint8_t*>(act),
+                 static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales), mu,
+                 static_cast<uint16_t*>(U_bf16), reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
+kq_status kq_debug_transform(const kq_layer_desc* desc, const void* weights, const void* X_bf16,
+                             int32_t M, float* Xt, float* mu, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (M <= 0 || !weights || !X_bf16 || !Xt || !mu) return KQ_ERR_INVALID_ARG;
+  if (!aligned(X_bf16) || !aligned(Xt) || !aligned(weights)) return KQ_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  QuantParams qp;
+  s = fill_quant_params(desc, weights, X_bf16, M, nullptr, &qp, di);
+  if (s != KQ_OK) return s;
+  // m_pad = M: no padding rows in debug mode; outputs go to the caller's arrays
+  qp.m_pad = M;
+  qp.codes = nullptr;
+  qp.sf = nullptr;
+  qp.mu = mu;
+  qp.xt = Xt;
+  qp.err = nullptr;
+  if (launch_quantize_rows(qp, true, di.sms, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
+kq_status kq_debug_encode_f32(const float* V, int32_t M, int32_t K, void* codes, void* scales,
+                              kq_stream_t stream) {
+  if (!V || !codes || !scales || M <= 0 || K <= 0) return KQ_ERR_INVALID_ARG;
+  if (K % 32 != 0) return KQ_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(V) & 15u) || (reinterpret_cast<uintptr_t>(codes) & 15u))
+    return KQ_ERR_ALIGNMENT;
+  DeviceInfo di;
+  kq_status s = current_device(&di);
+  if (s != KQ_OK) return s;
+  if (launch_encode_f32(V, M, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
+kq_status kq_last_device_error(const kq_layer_desc* desc, void* act, int32_t M, kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (!act || M <= 0) return KQ_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KQ_ERR_CUDA;
+  uint32_t word = 0;
+  const ActLayout AL = alayout(desc, M);
+  uint8_t* a = static_cast<uint8_t*>(act);
+  if (cudaMemcpy(&word, a + AL.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return KQ_ERR_CUDA;
+  if (word != 0 && cudaMemset(a + AL.err, 0, 4) != cudaSuccess) return KQ_ERR_CUDA;
+  return word ? KQ_ERR_DEVICE_TIMEOUT : KQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,62 @@
+// Internal declarations shared by the library's translation units: kernel parameter
+// blocks and launcher prototypes.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "encode.cuh"
+#include "layout.cuh"
+#include "sm100.cuh"
+
+namespace kq {
+
+struct QuantParams {
+  CUtensorMap tmap_x;          // X viewed as [M * K/32 lines, 32 bf16], 64-byte swizzle
+  float A[16];                 // Kronecker factor A (4x4, row-major)
+  float B[64];                 // Kronecker factor B (8x8, row-major)
+  int M, K, m_pad, kind, center;
+  int slots, warps_per_cta, ctas_per_sm, box_lines;
+  int64_t katoms;
+  uint8_t* codes;              // act codes [M, K/2]
+  uint8_t* sf;                 // act scales (tensor-core layout)
+  float* mu;                   // [m_pad]
+  const int32_t* perm;         // RPBH gather indices [K]
+  const float* sgn;            // RPBH sign / sqrt(32) [K]
+  float* xt;                   // debug: transformed values [M, K] (debug launch only)
+  uint32_t* err;
+};
+
+struct LowRankParams {
+  CUtensorMap tmap_x;          // X [M, K] bf16, box 64 x 128, 128-byte swizzle
+  CUtensorMap tmap_l1;         // [kUCols, K] bf16, box 64 x kUCols, 128-byte swizzle
+  const float* c1;             // [64]
+  uint16_t* u;                 // U [M, 64] bf16
+  int M, K, center;
+  uint32_t* err;
+};
+
+struct GemmParams {
+  CUtensorMap tmap_a;          // act codes [M, K/2] uint8, box 128 x 128, 128-byte swizzle
+  CUtensorMap tmap_b;          // residual codes [N, K/2] uint8, box 128 x BN
+  CUtensorMap tmap_u;          // U [M, 64] bf16, box 64 x 128
+  CUtensorMap tmap_l2;         // L2^T [N, 64] bf16, box 64 x BN
+  const uint8_t* sfa;          // act scales (tensor-core layout)
+  const uint8_t* sfb;          // residual scales (tensor-core layout, rows padded to 256)
+  const float* mu;             // [M] or null (no centring)
+  const float* s;              // [N]
+  void* y;                     // [M, N] f32 or bf16
+  int M, N, K, rank_pad;
+  int64_t katoms;
+  uint32_t* err;
+};
+
+cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sms,
+                                 cudaStream_t st);
+cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint8_t* scales,
+                              cudaStream_t st);
+cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st);
+cudaError_t launch_gemm(const GemmParams& p, int bn, bool out_bf16, cudaStream_t st);
+
+}  // namespace kq

@@ -1,0 +1,94 @@
+// Memory layouts of the prepared-weights buffer and of the activation workspace.
+//
+// Block scales (one E8M0 byte per 32 elements along K) are stored in the layout the
+// block-scaled tensor-core MMA consumes: rows are grouped by 128 and the K blocks by 4;
+// each (128-row group, 4-block group) is one 512-byte atom in which the byte of
+// (row r, block b) sits at  (r % 32) * 16 + ((r % 128) / 32) * 4 + (b % 4).
+// Atoms of one row group are consecutive along K, so the scales of one 128-row x
+// 256-element GEMM tile are one contiguous 1 KB run. The K-block count is padded to a
+// multiple of 8 (whole 256-element GEMM k-tiles); padding scales are written as 0.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+
+namespace kq {
+
+constexpr int kBlock = 32;          // MXFP4 block size along K
+constexpr int kTileK = 256;         // FP4 elements per GEMM k-tile (128 bytes per row)
+constexpr int kRankPad = 64;        // low-rank dimension as stored (rank <= 64)
+constexpr int kUCols = 2 * kRankPad + 16;   // U-kernel MMA width: L1' hi, L1' lo, ones row
+constexpr size_t kAlign = 1024;
+
+__host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ constexpr int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// number of 4-block atoms per 128-row group for a given K
+__host__ __device__ constexpr int64_t sf_katoms(int64_t K) { return 2 * cdiv(K, kTileK); }
+__host__ __device__ constexpr size_t sf_bytes(int64_t rows_pad, int64_t K) {
+  return static_cast<size_t>(rows_pad / 128) * static_cast<size_t>(sf_katoms(K)) * 512u;
+}
+__host__ __device__ __forceinline__ size_t sf_offset(int64_t row, int64_t kb, int64_t katoms) {
+  return static_cast<size_t>(row / 128) * static_cast<size_t>(katoms) * 512u +
+         static_cast<size_t>(kb / 4) * 512u + static_cast<size_t>(row % 32) * 16u +
+         static_cast<size_t>((row % 128) / 32) * 4u + static_cast<size_t>(kb % 4);
+}
+
+struct WeightsLayout {
+  int64_t K = 0, N = 0, rank = 0, rp = 0, n_pad = 0;
+  bool center = false;
+  int kind = 0;
+  size_t rcodes = 0;   // uint8 [N, K/2]     residual codes (R^T, K-major)
+  size_t rsf = 0;      // uint8 tiled        residual scales, rows padded to 256
+  size_t l2t = 0;      // bf16  [N, rp]      L2^T (K-major B operand of the low-rank MMA)
+  size_t l1t = 0;      // bf16  [kUCols, K]  rows 0..63 L1'^T hi, 64..127 lo, 128 ones
+  size_t c1 = 0;       // f32   [rp]         1^T (L1' hi + lo)
+  size_t s = 0;        // f32   [N]          1^T W
+  size_t perm = 0;     // int32 [K]          RPBH gather indices
+  size_t sgn = 0;      // f32   [K]          RPBH sign[k] / sqrt(32)
+  size_t total = 0;
+
+  __host__ __device__ static WeightsLayout make(int64_t K, int64_t N, int64_t rank, bool center,
+                                                int kind) {
+    WeightsLayout L;
+    L.K = K; L.N = N; L.rank = rank; L.rp = rank > 0 ? kRankPad : 0; L.center = center;
+    L.kind = kind;
+    L.n_pad = cdiv(N, 256) * 256;
+    size_t o = 256;  // header
+    L.rcodes = o; o = align_up(o + static_cast<size_t>(N) * (K / 2), kAlign);
+    L.rsf = o;    o = align_up(o + sf_bytes(L.n_pad, K), kAlign);
+    L.l2t = o;    o = align_up(o + static_cast<size_t>(N) * L.rp * 2, kAlign);
+    L.l1t = o;    o = align_up(o + (L.rp ? static_cast<size_t>(kUCols) * K * 2 : 0), kAlign);
+    L.c1 = o;     o = align_up(o + static_cast<size_t>(L.rp) * 4, kAlign);
+    L.s = o;      o = align_up(o + static_cast<size_t>(N) * 4, kAlign);
+    L.perm = o;   o = align_up(o + (kind == 2 ? static_cast<size_t>(K) * 4 : 0), kAlign);
+    L.sgn = o;    o = align_up(o + (kind == 2 ? static_cast<size_t>(K) * 4 : 0), kAlign);
+    L.total = o;
+    return L;
+  }
+};
+
+struct ActLayout {
+  int64_t M = 0, m_pad = 0, K = 0, rp = 0;
+  size_t err = 0;      // uint32 device error word
+  size_t codes = 0;    // uint8 [M, K/2]
+  size_t sf = 0;       // uint8 tiled, rows padded to 128
+  size_t mu = 0;       // f32 [m_pad]
+  size_t u = 0;        // bf16 [M, rp]
+  size_t total = 0;
+
+  __host__ __device__ static ActLayout make(int64_t M, int64_t K, int64_t rank) {
+    ActLayout L;
+    L.M = M; L.K = K; L.rp = rank > 0 ? kRankPad : 0;
+    L.m_pad = cdiv(M, 128) * 128;
+    size_t o = 0;
+    L.err = o;    o = 256;
+    L.codes = o;  o = align_up(o + static_cast<size_t>(M) * (K / 2), kAlign);
+    L.sf = o;     o = align_up(o + sf_bytes(L.m_pad, K), kAlign);
+    L.mu = o;     o = align_up(o + static_cast<size_t>(L.m_pad) * 4, kAlign);
+    L.u = o;      o = align_up(o + static_cast<size_t>(M) * L.rp * 2, kAlign);
+    L.total = o;
+    return L;
+  }
+};
+
+}  // namespace kq
