@@ -240,17 +240,10 @@ def main():
                      "Y": torch.empty((w.M, w.N), dtype=ydt, device=dev)})
     stream = torch.cuda.current_stream()
 
-    def step(j, ev=None):
+    def step(j):
         s = sets[j]
-        cur = torch.cuda.current_stream()
-        if ev is not None:
-            ev[0].record(cur)
         kq.quantize_act(L, s["w"], s["X"], s["act"])
-        if ev is not None:
-            ev[1].record(cur)
         kq.gemm(L, s["w"], s["act"], w.M, s["Y"], odt)
-        if ev is not None:
-            ev[2].record(cur)
 
     for i in range(args.warmup):
         step(i % R)
@@ -258,21 +251,41 @@ def main():
     for s in sets:
         assert kq.last_device_error(L, s["act"], w.M) == 0
 
-    # CUDA graph of one rotation (R steps) with per-phase events
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(R)]
-    graph = None
+    # CUDA graphs: one rotation (R steps) of the whole path, and phase-isolated rotations
+    # (quantize only, GEMM only) used to attribute the step time to kernels
+    graph = gq = gg = None
     if not args.no_graph:
         try:
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, capture_error_mode="relaxed"):
                 for j in range(R):
-                    step(j, evs[j])
+                    step(j)
+            gq = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gq, capture_error_mode="relaxed"):
+                for j in range(R):
+                    kq.quantize_act(L, sets[j]["w"], sets[j]["X"], sets[j]["act"])
+            gg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gg, capture_error_mode="relaxed"):
+                for j in range(R):
+                    kq.gemm(L, sets[j]["w"], sets[j]["act"], w.M, sets[j]["Y"], odt)
             graph.replay()
+            gq.replay()
+            gg.replay()
             torch.cuda.synchronize()
         except Exception as e:  # pragma: no cover - fall back to eager launches
             print(f"# graph capture failed ({e}); timing eager launches", file=sys.stderr)
-            graph = None
-            stream = torch.cuda.current_stream()
+            graph = gq = gg = None
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, n):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b)
 
     clocks = Clocks(local_rank)
     if world > 1:
@@ -288,12 +301,9 @@ def main():
             graph.replay()
         for j in range(rem):
             step(j)
-        # per-phase event times come from the last complete replay
-        if full == 0:
-            graph.replay()
     else:
         for i in range(args.steps):
-            step(i % R, evs[i % R])
+            step(i % R)
     t_end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
@@ -304,8 +314,14 @@ def main():
         elapsed_ms = float(t.item())
         dist.barrier()
 
-    q_ms = float(np.mean([evs[j][0].elapsed_time(evs[j][1]) for j in range(R)]))
-    g_ms = float(np.mean([evs[j][1].elapsed_time(evs[j][2]) for j in range(R)]))
+    # per-kernel attribution: the same launches, one phase at a time
+    reps = max(1, min(args.steps, 2000) // R)
+    if gq is not None:
+        q_ms = timed(gq.replay, reps) / (reps * R)
+        g_ms = timed(gg.replay, reps) / (reps * R)
+    else:
+        q_ms = timed(lambda: [kq.quantize_act(L, s["w"], s["X"], s["act"]) for s in sets], reps) / (reps * R)
+        g_ms = timed(lambda: [kq.gemm(L, s["w"], s["act"], w.M, s["Y"], odt) for s in sets], reps) / (reps * R)
     for s in sets:
         assert kq.last_device_error(L, s["act"], w.M) == 0
 
@@ -387,7 +403,8 @@ def main():
                    "out_dtype": args.out, "parallelism": f"replicas x{world} (token-sharded)",
                    "l2": f"{R} rotating buffer sets of {set_bytes / 1e6:.0f} MB (> L2)",
                    "graph": graph is not None},
-        "phases_ms": {"quantize": q_ms, "gemm": g_ms},
+        "phases_ms": {"quantize": q_ms, "gemm": g_ms,
+                      "how": "phase-isolated CUDA-graph replays over the same buffer sets"},
         "quantize_gbs": q_bytes / (q_ms * 1e-3) / 1e9,
         "gemm_tflops": gemm_flops / (g_ms * 1e-3) / 1e12,
         "roofline": roof,

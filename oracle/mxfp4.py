@@ -124,18 +124,23 @@ def decode(codes, scales) -> np.ndarray:
 
 
 def decision_margin(v) -> np.ndarray:
-    """Relative distance of each scaled element to its nearest rounding decision point
-    (a midpoint between grid values, or the block's scale change point amax = 2^k).
-    Used by tests to accept code differences that arise only from a last-ulp
-    difference in a float32 value computed in another order."""
+    """Distance of each element to its nearest rounding decision point, in units of its
+    block's maximum magnitude: min_i | |v| - mid_i * 2^e | / amax, where mid_i are the
+    midpoints between E2M1 grid values; and, for the whole block, the relative distance
+    of amax to the nearest power of two (where the shared scale changes).
+
+    Used by tests to accept code differences caused only by a last-ulp difference of a
+    float32 value computed in another order. The unit is the block maximum because that
+    is the unit in which a transform's rounding error is bounded (a Hadamard output can be
+    much smaller than its inputs)."""
     v = np.asarray(v, dtype=np.float64)
     blk = v.reshape(v.shape[:-1] + (v.shape[-1] // BLOCK, BLOCK))
     amax = np.max(np.abs(blk), axis=-1, keepdims=True)
     e = shared_exponent(amax[..., 0])[..., None]
-    w = np.abs(blk) / np.exp2(e.astype(np.float64))
+    scale = np.exp2(e.astype(np.float64))
+    w = np.abs(blk) / scale
     mids = (E2M1_MAGNITUDE[1:] + E2M1_MAGNITUDE[:-1]) / 2.0
-    d = np.min(np.abs(w[..., None] - mids), axis=-1) / np.maximum(w, 1e-300)
-    # amax near a power of two moves the whole block's scale
+    d = np.min(np.abs(w[..., None] - mids), axis=-1) * scale / np.maximum(amax, 1e-300)
     la = np.log2(np.maximum(amax, 1e-300))
     dscale = np.abs(la - np.rint(la)) * np.log(2.0)
     d = np.minimum(d, np.broadcast_to(dscale, d.shape))

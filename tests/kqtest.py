@@ -14,7 +14,7 @@ from synthetic import make_inputs, workload
 def pack_nibbles(codes: np.ndarray) -> np.ndarray:
     """uint8 codes [rows, K] (0..15) -> canonical [rows, K/2], element 2j in the low nibble."""
     c = np.asarray(codes, dtype=np.uint8)
-    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+    return np.ascontiguousarray((c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8))
 
 
 def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
