@@ -86,8 +86,23 @@ def test_quantize_act_matches_oracle(cuda_device, case):
     assert np.all(blk_margin[bad_s] < 2e-5)
     ok_blocks = np.repeat(~bad_s, 32, axis=1)
     bad_c = (gc != ref["codes"]) & ok_blocks
-    assert np.all(margin[bad_c] < 2e-5), (
-        f"{bad_c.sum()} code mismatches, max block-relative margin {margin[bad_c].max():.3e}")
+    if not np.all(margin[bad_c] < 2e-5):
+        # diagnostics: the same kernel's transform output (debug entry) at the mismatches
+        Xt = torch.empty((w.M, w.K), dtype=torch.float32, device="cuda")
+        mud = torch.empty((w.M,), dtype=torch.float32, device="cuda")
+        kq.debug_transform(L, wbuf, X, Xt, mud)
+        xt = Xt.cpu().double().numpy()
+        rr, cc = np.nonzero(bad_c & (margin >= 2e-5))
+        lines = []
+        for r_, c_ in list(zip(rr, cc))[:12]:
+            b_ = c_ // 32
+            blk = ref["Xt32"][r_, 32 * b_:32 * b_ + 32]
+            dc, _ = mxfp4.encode(xt[r_:r_ + 1, 32 * b_:32 * b_ + 32].astype(np.float32).astype(np.float64))
+            lines.append(f"row {r_} col {c_} (blk {b_}, lane-blk {b_ % 32}) oracle v={ref['Xt32'][r_, c_]:.6g} "
+                         f"gpu-debug v={xt[r_, c_]:.6g} amax={np.abs(blk).max():.4g} "
+                         f"code oracle={ref['codes'][r_, c_]} gpu={gc[r_, c_]} enc(debug)={dc[0, c_ % 32]}")
+        raise AssertionError(f"{bad_c.sum()} code mismatches away from a decision point:\n" +
+                             "\n".join(lines))
     assert bad_c.mean() < 1e-3
     np.testing.assert_allclose(mu.cpu().numpy(), ref["mu"], rtol=1e-6,
                                atol=1e-6 * (np.abs(ref["mu"]).max() + 1.0))
