@@ -85,7 +85,10 @@ def test_quantize_act_matches_oracle(cuda_device, case):
     blk_margin = margin.reshape(w.M, -1, 32).min(axis=2)
     assert np.all(blk_margin[bad_s] < 2e-5)
     ok_blocks = np.repeat(~bad_s, 32, axis=1)
-    bad_c = (gc != ref["codes"]) & ok_blocks
+    # +0 (0x0) and -0 (0x8) decode to the same value: where the transform cancels exactly,
+    # the sign of the zero is an artefact of summation order (fp32 kernel vs fp64 oracle)
+    canon = lambda c: np.where((c & 7) == 0, 0, c)
+    bad_c = (canon(gc) != canon(ref["codes"])) & ok_blocks
     if not np.all(margin[bad_c] < 2e-5):
         # diagnostics: the same kernel's transform output (debug entry) at the mismatches
         Xt = torch.empty((w.M, w.K), dtype=torch.float32, device="cuda")
