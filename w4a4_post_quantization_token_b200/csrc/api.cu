@@ -159,12 +159,6 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   const WeightsLayout WL = wlayout(d);
   const ActLayout AL = alayout(d, M);
   const int K = d->K, nb = K / kBlock;
-  int box_lines = 1;
-  for (int c = 1; c <= 256 && c <= nb; ++c) if (nb % c == 0) box_lines = c;
-  if (!make_tmap(&p->tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, 32,
-                 static_cast<uint64_t>(M) * nb, 64, 32, static_cast<uint32_t>(box_lines),
-                 CU_TENSOR_MAP_SWIZZLE_64B))
-    return KQ_ERR_CUDA;
   if (d->t.kind == KQ_T_KRON) {
     for (int i = 0; i < 16; ++i) p->A[i] = d->t.A[i];
     for (int i = 0; i < 64; ++i) p->B[i] = d->t.B[i];
@@ -172,20 +166,33 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   p->M = M; p->K = K; p->m_pad = static_cast<int>(AL.m_pad);
   p->kind = d->t.kind; p->center = d->center;
   p->katoms = sf_katoms(K);
-  p->box_lines = box_lines;
-  const size_t slot = align_up(static_cast<size_t>(K) * 2, 1024);
-  const size_t budget = 200 * 1024;
-  int nw = 8, slots = 2;
-  while (nw * slots * slot > budget && slots > 1) --slots;
-  while (nw * slots * slot > budget && nw > 1) nw >>= 1;
-  if (nw * slots * slot > budget) return KQ_ERR_UNSUPPORTED_SHAPE;
-  p->warps_per_cta = nw;
-  p->slots = slots;
-  const size_t smem = 1024 + static_cast<size_t>(nw) * slots * slot;
-  int per_sm = static_cast<int>((227 * 1024) / (smem + 1024));
-  if (per_sm < 1) per_sm = 1;
-  if (per_sm * nw > 32) per_sm = 32 / nw > 0 ? 32 / nw : 1;   // at most 32 warps per SM
-  p->ctas_per_sm = per_sm;
+  // groups of R rows, one thread per 32-element block
+  int R = static_cast<int>(cdiv(256, nb));
+  const int r_mem = static_cast<int>(32768 / (static_cast<size_t>(K) * 2));
+  if (R > r_mem) R = r_mem;
+  if (R > 64) R = 64;
+  if (R < 1) R = 1;
+  const int items = R * nb;
+  int box = 1;
+  for (int c = 1; c <= 256 && c <= items; ++c) if (items % c == 0) box = c;
+  p->rows_per_group = R;
+  p->box_lines = box;
+  if (!make_tmap(&p->tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, 32,
+                 static_cast<uint64_t>(M) * nb, 64, 32, static_cast<uint32_t>(box),
+                 CU_TENSOR_MAP_SWIZZLE_64B))
+    return KQ_ERR_CUDA;
+  const int nb_pad = static_cast<int>(p->katoms) * 4;
+  size_t off = 1024 + align_up(static_cast<size_t>(R) * nb_pad, 16) + static_cast<size_t>(items) * 4;
+  p->tables_off = align_up(off, 128);
+  const size_t tables = d->t.kind == KQ_T_RPBH ? static_cast<size_t>(K) * 2 + static_cast<size_t>(nb) * 4 : 0;
+  p->bufs_off = align_up(p->tables_off + tables, 1024);
+  const size_t buf_bytes = align_up(static_cast<size_t>(items) * 64, 1024);
+  const size_t budget = 227 * 1024;
+  if (p->bufs_off + buf_bytes > budget) return KQ_ERR_UNSUPPORTED_SHAPE;
+  p->nbufs = static_cast<int>((budget - p->bufs_off) / buf_bytes);
+  if (p->nbufs > 4) p->nbufs = 4;
+  p->smem_bytes = p->bufs_off + static_cast<size_t>(p->nbufs) * buf_bytes;
+  if (d->t.kind == KQ_T_RPBH && K > 65536) return KQ_ERR_UNSUPPORTED_SHAPE;
   (void)di;
   if (act) {
     p->codes = act + AL.codes;
@@ -227,12 +234,13 @@ kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* 
 }
 
 kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* act, int M, void* Y,
-                   int out_dtype, cudaStream_t st) {
+                   int out_dtype, cudaStream_t st, const DeviceInfo& di) {
   const WeightsLayout WL = wlayout(d);
   const ActLayout AL = alayout(d, M);
   const uint8_t* w = static_cast<const uint8_t*>(weights);
   const int K = d->K, N = d->N;
-  const int bn = (N % 256 == 0) ? 256 : (N % 128 == 0 ? 128 : 256);
+  const uint32_t bn = static_cast<uint32_t>(gemm_tile_n());
+  const bool bf16 = out_dtype == KQ_OUT_BF16;
   GemmParams gp;
   std::memset(&gp, 0, sizeof(gp));
   if (!make_tmap(&gp.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, act + AL.codes, static_cast<uint64_t>(K / 2),
@@ -240,18 +248,22 @@ kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* a
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return KQ_ERR_CUDA;
   if (!make_tmap(&gp.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w + WL.rcodes, static_cast<uint64_t>(K / 2),
-                 static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), 128,
-                 static_cast<uint32_t>(bn), CU_TENSOR_MAP_SWIZZLE_128B))
+                 static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), 128, bn,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
     return KQ_ERR_CUDA;
   if (d->rank > 0) {
     if (!make_tmap(&gp.tmap_u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act + AL.u, kRankPad,
                    static_cast<uint64_t>(M), kRankPad * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return KQ_ERR_CUDA;
     if (!make_tmap(&gp.tmap_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w + WL.l2t, kRankPad,
-                   static_cast<uint64_t>(N), kRankPad * 2, 64, static_cast<uint32_t>(bn),
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+                   static_cast<uint64_t>(N), kRankPad * 2, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))
       return KQ_ERR_CUDA;
   }
+  if (!make_tmap(&gp.tmap_y, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                 Y, static_cast<uint64_t>(N), static_cast<uint64_t>(M),
+                 static_cast<uint64_t>(N) * (bf16 ? 2 : 4), bf16 ? 64 : 32, 32,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return KQ_ERR_CUDA;
   gp.sfa = act + AL.sf;
   gp.sfb = w + WL.rsf;
   gp.mu = d->center ? reinterpret_cast<const float*>(act + AL.mu) : nullptr;
@@ -261,7 +273,7 @@ kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* a
   gp.rank_pad = d->rank > 0 ? kRankPad : 0;
   gp.katoms = sf_katoms(K);
   gp.err = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(act) + AL.err);
-  if (launch_gemm(gp, bn, out_dtype == KQ_OUT_BF16, st) != cudaSuccess) return KQ_ERR_CUDA;
+  if (launch_gemm(gp, bf16, di.sms, st) != cudaSuccess) return KQ_ERR_CUDA;
   return KQ_OK;
 }
 
@@ -369,7 +381,7 @@ kq_status kq_gemm(const kq_layer_desc* desc, const void* weights, const void* ac
   DeviceInfo di;
   if ((s = current_device(&di)) != KQ_OK) return s;
   return run_gemm(desc, weights, static_cast<const uint8_t*>(act), M, Y, out_dtype,
-                  reinterpret_cast<cudaStream_t>(stream));
+                  reinterpret_cast<cudaStream_t>(stream), di);
 }
 
 kq_status kq_linear(const kq_layer_desc* desc, const void* weights, const void* X_bf16, int32_t M,
@@ -381,8 +393,10 @@ kq_status kq_linear(const kq_layer_desc* desc, const void* weights, const void* 
   if (!aligned(Y)) return KQ_ERR_ALIGNMENT;
   s = kq_quantize_act(desc, weights, X_bf16, M, act, act_bytes, stream);
   if (s != KQ_OK) return s;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
   return run_gemm(desc, weights, static_cast<const uint8_t*>(act), M, Y, out_dtype,
-                  reinterpret_cast<cudaStream_t>(stream));
+                  reinterpret_cast<cudaStream_t>(stream), di);
 }
 
 kq_status kq_linear_host(const kq_layer_desc* desc, const void* weights, const void* X_host,

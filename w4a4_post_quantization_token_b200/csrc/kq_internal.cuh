@@ -17,7 +17,8 @@ struct QuantParams {
   float A[16];                 // Kronecker factor A (4x4, row-major)
   float B[64];                 // Kronecker factor B (8x8, row-major)
   int M, K, m_pad, kind, center;
-  int slots, warps_per_cta, ctas_per_sm, box_lines;
+  int rows_per_group, box_lines, nbufs;
+  size_t tables_off, bufs_off, smem_bytes;   // dynamic shared memory carve-up
   int64_t katoms;
   uint8_t* codes;              // act codes [M, K/2]
   uint8_t* sf;                 // act scales (tensor-core layout)
@@ -42,8 +43,9 @@ struct GemmParams {
   CUtensorMap tmap_b;          // residual codes [N, K/2] uint8, box 128 x BN
   CUtensorMap tmap_u;          // U [M, 64] bf16, box 64 x 128
   CUtensorMap tmap_l2;         // L2^T [N, 64] bf16, box 64 x BN
+  CUtensorMap tmap_y;          // Y [M, N] f32 or bf16, box (128 bytes) x 32 rows, 128-byte swizzle
   const uint8_t* sfa;          // act scales (tensor-core layout)
-  const uint8_t* sfb;          // residual scales (tensor-core layout, rows padded to 256)
+  const uint8_t* sfb;          // residual scales (tensor-core layout, one spare row atom)
   const float* mu;             // [M] or null (no centring)
   const float* s;              // [N]
   void* y;                     // [M, N] f32 or bf16
@@ -57,6 +59,7 @@ cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sm
 cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint8_t* scales,
                               cudaStream_t st);
 cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st);
-cudaError_t launch_gemm(const GemmParams& p, int bn, bool out_bf16, cudaStream_t st);
+cudaError_t launch_gemm(const GemmParams& p, bool out_bf16, int num_sms, cudaStream_t st);
+int gemm_tile_n();
 
 }  // namespace kq

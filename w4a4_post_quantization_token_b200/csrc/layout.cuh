@@ -38,7 +38,7 @@ struct WeightsLayout {
   bool center = false;
   int kind = 0;
   size_t rcodes = 0;   // uint8 [N, K/2]     residual codes (R^T, K-major)
-  size_t rsf = 0;      // uint8 tiled        residual scales, rows padded to 256
+  size_t rsf = 0;      // uint8 tiled        residual scales, rows padded (see n_pad)
   size_t l2t = 0;      // bf16  [N, rp]      L2^T (K-major B operand of the low-rank MMA)
   size_t l1t = 0;      // bf16  [kUCols, K]  rows 0..63 L1'^T hi, 64..127 lo, 128 ones
   size_t c1 = 0;       // f32   [rp]         1^T (L1' hi + lo)
@@ -52,7 +52,9 @@ struct WeightsLayout {
     WeightsLayout L;
     L.K = K; L.N = N; L.rank = rank; L.rp = rank > 0 ? kRankPad : 0; L.center = center;
     L.kind = kind;
-    L.n_pad = cdiv(N, 256) * 256;
+    // 192-wide GEMM tiles read two 128-row scale atoms starting at floor(n0 / 128): keep one
+    // spare (zero) atom after the last real one
+    L.n_pad = cdiv(N, 128) * 128 + 128;
     size_t o = 256;  // header
     L.rcodes = o; o = align_up(o + static_cast<size_t>(N) * (K / 2), kAlign);
     L.rsf = o;    o = align_up(o + sf_bytes(L.n_pad, K), kAlign);

@@ -1,10 +1,10 @@
 // Online half of the W4A4 linear layer: per-token centring, block transform and
 // MXFP4 encoding of bf16 activations, plus the low-rank input U on the tensor cores.
 //
-//  * k_quantize_rows -- one warp per token row. The row is staged in shared memory by a
-//    TMA tensor load with the 64-byte swizzle (each 32-element block is one 64-byte line,
-//    its four 16-byte chunks permuted by line), so that one thread per block reads its
-//    block without bank conflicts. Centring (CentriQ abstract: centre each token before
+//  * k_quantize_rows -- groups of R token rows per CTA step, one thread per 32-element
+//    block. Rows are staged in shared memory by a TMA tensor load with the 64-byte swizzle
+//    (each block is one 64-byte line, its four 16-byte chunks permuted by line), so that
+//    one thread per block reads its block without bank conflicts. Centring (CentriQ abstract: centre each token before
 //    the rotation) uses an fp32 per-block sum and an fp64 cross-block sum, then
 //    x - mu as (x - mu_hi) - mu_lo in fp32. The block transform runs in registers:
 //    Kronecker A^T X_m B with A, B as kernel parameters (KroQuant commentary, section 02),
@@ -109,137 +109,184 @@ __device__ __forceinline__ void fwht32(float (&v)[32]) {
 // ----------------------------------------------------------------------------------
 // k_quantize_rows
 // ----------------------------------------------------------------------------------
+// One CTA processes groups of R consecutive token rows; one thread per 32-element block
+// (R * K/32 threads). Groups are staged by TMA (64-byte swizzle, one 64-byte line per
+// block) into a ring of up to 4 slots; the CTA walks groups blockIdx.x, +gridDim.x, ...
+constexpr int kQMaxBufs = 4;
+
 template <int KIND, bool CENTER, bool DEBUG_XT>
-__global__ void __launch_bounds__(256) k_quantize_rows(const __grid_constant__ QuantParams p) {
+__global__ void __launch_bounds__(512, 1) k_quantize_rows(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int NW = blockDim.x >> 5;
-  const int S = p.slots;
-  const uint32_t row_bytes = static_cast<uint32_t>(p.K) * 2u;
-  const uint32_t slot_bytes = static_cast<uint32_t>(align_up(row_bytes, 1024));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem);
-  uint8_t* bufs = smem + 1024;
-  uint8_t* mybuf = bufs + static_cast<size_t>(warp) * S * slot_bytes;
-  uint64_t* mybar = bars + warp * S;
+  const int tid = threadIdx.x;
   const int nb = p.K / kBlock;
   const int nb_pad = static_cast<int>(p.katoms) * 4;
-  const int TW = gridDim.x * NW;
-  const int gw = blockIdx.x * NW + warp;
+  const int R = p.rows_per_group;
+  const int items = R * nb;
+  const uint32_t grp_bytes = static_cast<uint32_t>(items) * 64u;
+  const uint32_t buf_bytes = static_cast<uint32_t>(align_up(grp_bytes, 1024));
+  // shared memory carve-up
+  const int nbufs = p.nbufs;                                                 // <= kQMaxBufs
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);                       // [nbufs]
+  float2* mus = reinterpret_cast<float2*>(smem + 64);                       // [R] (hi, lo)
+  uint8_t* sst = smem + 64 + 8 * 64;                                        // scale staging
+  float* bsum = reinterpret_cast<float*>(smem + 1024 + align_up(static_cast<size_t>(R) * nb_pad, 16));
+  uint8_t* tables = smem + p.tables_off;                                    // RPBH tables
+  uint8_t* bufs = smem + p.bufs_off;
 
-  if (lane == 0) {
-    for (int s = 0; s < S; ++s) mbar_init(&mybar[s], 1);
+  const int ngroups = static_cast<int>(cdiv(p.M, R));
+  if (tid == 0) {
+    for (int b = 0; b < nbufs; ++b) mbar_init(&full[b], 1);
     fence_mbar_init();
     prefetch_tmap(&p.tmap_x);
   }
-  __syncwarp();
+  if (KIND == 2) {
+    // perm as uint16, block b's 32 entries (64 bytes) with 16-byte chunks swizzled like the rows;
+    // sign bits: one 32-bit word per block
+    uint16_t* pt = reinterpret_cast<uint16_t*>(tables);
+    uint32_t* sb = reinterpret_cast<uint32_t*>(tables + static_cast<size_t>(p.K) * 2);
+    for (int k = tid; k < p.K; k += blockDim.x) {
+      const uint32_t off = static_cast<uint32_t>(k) * 2u;
+      pt[swz64(off) / 2] = static_cast<uint16_t>(p.perm[k]);
+    }
+    for (int b = tid; b < nb; b += blockDim.x) {
+      uint32_t w = 0;
+      for (int j = 0; j < 32; ++j) w |= (p.sgn[32 * b + j] < 0.f ? 1u : 0u) << j;
+      sb[b] = w;
+    }
+  }
+  __syncthreads();
 
-  // one row = nb 64-byte lines, loaded in boxes of up to 256 lines
-  auto issue = [&](int row, int s) {
-    uint8_t* dst = mybuf + static_cast<size_t>(s) * slot_bytes;
-    mbar_arrive_expect_tx(&mybar[s], row_bytes);
-    for (int l0 = 0; l0 < nb; l0 += p.box_lines)
-      tma_load_2d(dst + static_cast<size_t>(l0) * 64u, &p.tmap_x, 0,
-                  row * nb + l0, &mybar[s]);
+  auto issue = [&](int g, int buf) {
+    uint8_t* dst = bufs + static_cast<size_t>(buf) * buf_bytes;
+    mbar_arrive_expect_tx(&full[buf], grp_bytes);
+    const int l0 = g * items;
+    for (int l = 0; l < items; l += p.box_lines)
+      tma_load_2d(dst + static_cast<size_t>(l) * 64u, &p.tmap_x, 0, l0 + l, &full[buf]);
   };
-  if (lane == 0)
-    for (int s = 0; s < S; ++s) {
-      const int row = gw + s * TW;
-      if (row < p.M) issue(row, s);
+  if (tid == 0)
+    for (int b = 0; b < nbufs; ++b) {
+      const int g = blockIdx.x + b * gridDim.x;
+      if (g < ngroups) issue(g, b);
     }
 
-  for (int i = 0;; ++i) {
-    const int row = gw + i * TW;
-    if (row >= p.m_pad) break;
-    if (row >= p.M) {
-      // padding row of the last 128-row group: zero scales so the GEMM sees finite values
-      if (!DEBUG_XT) {
-        for (int b4 = lane * 4; b4 < nb_pad; b4 += 128)
-          *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, b4, p.katoms)) = 0u;
-        if (lane == 0) p.mu[row] = 0.f;
-      }
-      continue;
-    }
-    const int s = i % S;
-    const uint32_t parity = static_cast<uint32_t>(i / S) & 1u;
-    if (!mbar_wait(&mybar[s], parity, p.err, KQ_DEV_ERR_TIMEOUT_FULL)) break;
-    const uint8_t* rowbuf = mybuf + static_cast<size_t>(s) * slot_bytes;
+  int iter = 0;
+  for (int g = blockIdx.x; g < ngroups; g += gridDim.x, ++iter) {
+    const int buf = iter % nbufs;
+    const uint32_t parity = static_cast<uint32_t>(iter / nbufs) & 1u;
+    const int row0 = g * R;
+    __syncthreads();   // previous group's staging reads are done
+    const bool ok = __syncthreads_and(mbar_wait(&full[buf], parity, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
+    if (!ok) break;
+    const uint8_t* gbuf = bufs + static_cast<size_t>(buf) * buf_bytes;
 
-    float mu_hi = 0.f, mu_lo = 0.f;
     if (CENTER) {
-      double part = 0.0;
-      for (int b = lane; b < nb; b += 32) {
+      for (int i = tid; i < items; i += blockDim.x) {
         float v[32];
-        load_block_swz(rowbuf, b, v);
-        part += static_cast<double>(tree_sum32(v));
+        load_block_swz(gbuf, i, v);
+        bsum[i] = tree_sum32(v);
       }
-      const double mu64 = warp_sum_f64(part) / static_cast<double>(p.K);
-      mu_hi = static_cast<float>(mu64);
-      mu_lo = static_cast<float>(mu64 - static_cast<double>(mu_hi));
-      if (lane == 0) p.mu[row] = mu_hi;
-    } else if (lane == 0) {
-      p.mu[row] = 0.f;
+      __syncthreads();
+      const int warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
+      for (int r = warp; r < R; r += nwarps) {
+        double part = 0.0;
+        for (int b = lane; b < nb; b += 32) part += static_cast<double>(bsum[r * nb + b]);
+        const double mu64 = warp_sum_f64(part) / static_cast<double>(p.K);
+        const float hi = static_cast<float>(mu64);
+        const float lo = static_cast<float>(mu64 - static_cast<double>(hi));
+        if (lane == 0) {
+          mus[r] = make_float2(hi, lo);
+          if (row0 + r < p.M) p.mu[row0 + r] = hi;
+        }
+      }
+      __syncthreads();
+    } else if (tid < R && row0 + tid < p.M) {
+      p.mu[row0 + tid] = 0.f;
     }
 
-    const int iters = (nb_pad + 31) / 32;
-    for (int it = 0; it < iters; ++it) {
-      const int b = it * 32 + lane;
-      uint32_t sb = 0;
-      if (b < nb) {
-        float v[32];
-        if (KIND == 2) {
-          const int4* pp = reinterpret_cast<const int4*>(p.perm + b * kBlock);
+    for (int i = tid; i < items; i += blockDim.x) {
+      const int r = i / nb, b = i - r * nb;
+      const int row = row0 + r;
+      if (row >= p.M) continue;
+      float v[32];
+      // swizzle positions are taken relative to the 1024-byte aligned ring slot: line index
+      // i = r * nb + b for the block, element index r * K + e for a gathered element
+      if (KIND == 2) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const int4 ix = __ldg(pp + q);
-            v[4 * q + 0] = load_elem_swz(rowbuf, ix.x);
-            v[4 * q + 1] = load_elem_swz(rowbuf, ix.y);
-            v[4 * q + 2] = load_elem_swz(rowbuf, ix.z);
-            v[4 * q + 3] = load_elem_swz(rowbuf, ix.w);
-          }
-        } else {
-          load_block_swz(rowbuf, b, v);
-        }
-        if (CENTER) {
+        for (int c = 0; c < 4; ++c) {
+          const uint4 ix = *reinterpret_cast<const uint4*>(
+              tables + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
+          const uint32_t w4[4] = {ix.x, ix.y, ix.z, ix.w};
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = (v[j] - mu_hi) - mu_lo;
-        }
-        if (KIND == 1) {
-          kron_apply(v, p.A, p.B);
-        } else if (KIND == 2) {
-          fwht32(v);
-          const float4* sg = reinterpret_cast<const float4*>(p.sgn + b * kBlock);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 g = __ldg(sg + q);
-            v[4 * q + 0] *= g.x; v[4 * q + 1] *= g.y;
-            v[4 * q + 2] *= g.z; v[4 * q + 3] *= g.w;
+          for (int t = 0; t < 4; ++t) {
+            v[8 * c + 2 * t] = load_elem_swz(gbuf, r * p.K + static_cast<int>(w4[t] & 0xFFFFu));
+            v[8 * c + 2 * t + 1] = load_elem_swz(gbuf, r * p.K + static_cast<int>(w4[t] >> 16));
           }
         }
-        if (DEBUG_XT) {
-          float4* o = reinterpret_cast<float4*>(p.xt + static_cast<size_t>(row) * p.K + b * kBlock);
-#pragma unroll
-          for (int q = 0; q < 8; ++q)
-            o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-        } else {
-          uint32_t c[4];
-          sb = mx_encode32(v, c);
-          *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + b * 16) =
-              make_uint4(c[0], c[1], c[2], c[3]);
-        }
+      } else {
+        load_block_swz(gbuf, i, v);
       }
-      if (!DEBUG_XT) {
-        const uint32_t w = sb | (__shfl_down_sync(0xffffffffu, sb, 1) << 8) |
-                           (__shfl_down_sync(0xffffffffu, sb, 2) << 16) |
-                           (__shfl_down_sync(0xffffffffu, sb, 3) << 24);
-        if ((lane & 3) == 0 && b < nb_pad)
-          *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, b, p.katoms)) = w;
+      if (CENTER) {
+        const float2 m = mus[r];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] = (v[j] - m.x) - m.y;
+      }
+      if (KIND == 1) {
+        kron_apply(v, p.A, p.B);
+      } else if (KIND == 2) {
+        fwht32(v);
+        const uint32_t sbits = reinterpret_cast<const uint32_t*>(tables + static_cast<size_t>(p.K) * 2)[b];
+        const float rs = 0.17677669529663687f;   // 1 / sqrt(32)
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          v[j] = __uint_as_float(__float_as_uint(v[j] * rs) ^ (((sbits >> j) & 1u) << 31));
+      }
+      if (DEBUG_XT) {
+        float4* o = reinterpret_cast<float4*>(p.xt + static_cast<size_t>(row) * p.K + b * kBlock);
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+          o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
+        uint32_t c[4];
+        const uint32_t sbyte = mx_encode32(v, c);
+        *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + b * 16) =
+            make_uint4(c[0], c[1], c[2], c[3]);
+        sst[r * nb_pad + b] = static_cast<uint8_t>(sbyte);
       }
     }
-    __syncwarp();
-    const int nrow = row + S * TW;
-    if (lane == 0 && nrow < p.M) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(nrow, s);
+    __syncthreads();   // all reads of this ring slot and all staged scales are done
+    if (tid == 0) {
+      const int gn = g + nbufs * gridDim.x;
+      if (gn < ngroups) {
+        fence_async_smem();
+        issue(gn, buf);
+      }
+    }
+    if (!DEBUG_XT) {
+      // scale words: 4 consecutive blocks of one row per 32-bit word, padding blocks = 0
+      const int wpr = nb_pad / 4;
+      for (int i = tid; i < R * wpr; i += blockDim.x) {
+        const int r = i / wpr, w = i - r * wpr;
+        const int row = row0 + r;
+        if (row >= p.M) continue;
+        uint32_t word = 0;
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int b = 4 * w + t;
+          const uint32_t v = b < nb ? sst[r * nb_pad + b] : 0u;
+          word |= v << (8 * t);
+        }
+        *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, 4 * w, p.katoms)) = word;
+      }
+    }
+  }
+  // rows M .. m_pad-1 of the last 128-row group: zero scales (finite values for the GEMM)
+  if (!DEBUG_XT) {
+    const int wpr = nb_pad / 4;
+    const int pad_rows = p.m_pad - p.M;
+    for (int i = blockIdx.x * blockDim.x + tid; i < pad_rows * wpr; i += gridDim.x * blockDim.x) {
+      const int r = p.M + i / wpr, w = i % wpr;
+      *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, 4 * w, p.katoms)) = 0u;
+      if (w == 0) p.mu[r] = 0.f;
     }
   }
 }
@@ -398,21 +445,20 @@ static cudaError_t launch_rows_t(const QuantParams& p, int num_sms, int block, s
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, block, smem);
   if (e != cudaSuccess) return e;
   if (per_sm < 1) per_sm = 1;
-  if (per_sm > p.ctas_per_sm) per_sm = p.ctas_per_sm;
-  // persistent warps: at most one resident wave; each warp walks rows with a grid stride
-  int64_t grid = cdiv(p.m_pad, block / 32);
-  const int64_t cap = static_cast<int64_t>(num_sms) * per_sm;
-  if (grid > cap) grid = cap;
+  const int64_t groups = cdiv(p.M, p.rows_per_group);
+  int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
+  if (grid > groups) grid = groups;
+  if (grid < 1) grid = 1;
   fn<<<static_cast<unsigned>(grid), block, smem, st>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sms,
                                  cudaStream_t st) {
-  const uint32_t slot = static_cast<uint32_t>(align_up(static_cast<size_t>(p.K) * 2, 1024));
-  const int NW = p.warps_per_cta;
-  const size_t smem = 1024 + static_cast<size_t>(NW) * p.slots * slot;
-  const int block = 32 * NW;
+  const int items = p.rows_per_group * (p.K / kBlock);
+  int block = static_cast<int>(align_up(static_cast<size_t>(items), 32));
+  if (block > 512) block = 512;
+  const size_t smem = p.smem_bytes;
   const int kind = p.kind, c = p.center ? 1 : 0;
 #define KQ_DISPATCH(KD, C)                                                             \
   if (kind == KD && c == C)                                                            \
