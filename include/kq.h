@@ -9,7 +9,9 @@
  *   Y     = deq(Q(Xt)) deq(Q(R)) + U L2 + mu s  (MXFP4 GEMM + low-rank + rank-1 branches)
  *
  * with, prepared once per layer: W' = P^-1 W, W' ~ L1 L2 (rank r, bf16 factors),
- * R = W' - L1 L2 in MXFP4, s = 1^T W, and online U = Xt L1.
+ * R = W' - L1 L2 in MXFP4, s = 1^T W, and online U = Xt L1. The low-rank branch runs in
+ * 16 bits: U is held as fp16 (saturated at +-65504) and multiplied with L2 (bf16 values,
+ * held as fp16) on the tensor cores with fp32 accumulation.
  *
  * Sources (commentary pages on the methods):
  *   - KroQuant: Kronecker-Structured Block Transforms for Efficient Post-Training
@@ -107,7 +109,8 @@ typedef struct {
 size_t kq_weights_bytes(const kq_layer_desc *desc);
 
 /* Bytes of the activation workspace for M tokens: MXFP4 codes, block scales in the
- * tensor-core layout, token means, low-rank activations U, and the device error word. */
+ * tensor-core layout, token means, low-rank activations U (fp16), and a small header
+ * holding the device error word. */
 size_t kq_act_bytes(const kq_layer_desc *desc, int32_t M);
 
 /* ---------------------------------------------------------------------------------
@@ -182,14 +185,15 @@ kq_status kq_weights_unpack(const kq_layer_desc *desc, const void *weights, void
                             kq_stream_t stream);
 
 /* Fill an activation workspace from canonical parts (mu may be null when centring is
- * off; U_bf16 [M, rank] may be null when rank == 0). */
+ * off; U_f16, the low-rank activations as fp16 [M, rank], may be null when rank == 0). */
 kq_status kq_act_pack(const kq_layer_desc *desc, const void *codes, const void *scales,
-                      const float *mu, const void *U_bf16, int32_t M, void *act,
+                      const float *mu, const void *U_f16, int32_t M, void *act,
                       size_t act_bytes, kq_stream_t stream);
 
-/* Read an activation workspace back into canonical parts (null pointers skip). */
+/* Read an activation workspace back into canonical parts (null pointers skip).
+ * U_f16 receives fp16 [M, rank]. */
 kq_status kq_act_unpack(const kq_layer_desc *desc, const void *act, int32_t M, void *codes,
-                        void *scales, float *mu, void *U_bf16, kq_stream_t stream);
+                        void *scales, float *mu, void *U_f16, kq_stream_t stream);
 
 /* ---------------------------------------------------------------------------------
  * Debug entry points (each runs one stage of the online half in isolation).

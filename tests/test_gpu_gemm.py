@@ -28,7 +28,7 @@ def _run(M, K, N, rank=0, center=False, out_bf16=False, seed=0):
     s = rng.standard_normal(N).astype(np.float32)
     mu = rng.standard_normal(M).astype(np.float32) * 3 if center else None
     if rank:
-        U = torch.randn(M, rank, dtype=torch.float32).to(torch.bfloat16)
+        U = torch.randn(M, rank, dtype=torch.float32).to(torch.float16)
         L2 = torch.randn(rank, N, dtype=torch.float32).to(torch.bfloat16)
         L1p = torch.zeros(K, rank, dtype=torch.float32)
     else:

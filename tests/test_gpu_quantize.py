@@ -5,7 +5,7 @@
 * the full quantize kernel (kq_quantize_act): MXFP4 codes/scales equal to the oracle's
   except where the oracle's float32 value sits within 2e-5 of a rounding decision point,
   measured in units of its block's maximum (the unit of the transform's error bound);
-  token means; low-rank input U within bf16 rounding."""
+  token means; low-rank input U within fp16 rounding."""
 import numpy as np
 import pytest
 
@@ -72,7 +72,7 @@ def test_quantize_act_matches_oracle(cuda_device, case):
     codes = torch.empty((w.M, w.K // 2), dtype=torch.uint8, device="cuda")
     scales = torch.empty((w.M, w.K // 32), dtype=torch.uint8, device="cuda")
     mu = torch.empty((w.M,), dtype=torch.float32, device="cuda")
-    U = torch.empty((w.M, max(w.rank, 1)), dtype=torch.bfloat16, device="cuda")
+    U = torch.empty((w.M, max(w.rank, 1)), dtype=torch.float16, device="cuda")
     kq.act_unpack(L, act, w.M, codes, scales, mu, U if w.rank else None)
     assert kq.last_device_error(L, act, w.M) == 0
     ref = olayer.quantize_act(inp["X"], inp["T"], w.center, prep)
@@ -113,7 +113,8 @@ def test_quantize_act_matches_oracle(cuda_device, case):
         Ug = U.float().cpu().double().numpy()
         Ur = ref["U"]
         rms = np.sqrt(np.mean(Ur ** 2))
-        assert np.all(np.abs(Ug - Ur) <= 2.0 ** -8 * np.abs(Ur) + 1e-3 * rms)
+        # fp16 rounding (2^-11 relative) plus the hi/lo bf16 representation of L1'
+        assert np.all(np.abs(Ug - Ur) <= 2.0 ** -10 * np.abs(Ur) + 1e-4 * rms)
 
 
 def test_quantize_is_deterministic(cuda_device):

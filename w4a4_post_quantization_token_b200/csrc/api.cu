@@ -160,39 +160,62 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   const ActLayout AL = alayout(d, M);
   const int K = d->K, nb = K / kBlock;
   if (d->t.kind == KQ_T_KRON) {
-    for (int i = 0; i < 16; ++i) p->A[i] = d->t.A[i];
-    for (int i = 0; i < 64; ++i) p->B[i] = d->t.B[i];
+    auto pair = [](float lo, float hi) {
+      uint32_t a, b;
+      std::memcpy(&a, &lo, 4);
+      std::memcpy(&b, &hi, 4);
+      return (static_cast<uint64_t>(b) << 32) | a;
+    };
+    for (int i = 0; i < 4; ++i)
+      for (int k = 0; k < 4; ++k) p->Ap[4 * i + k] = pair(d->t.A[4 * i + k], d->t.A[4 * i + k]);
+    for (int j = 0; j < 8; ++j)
+      for (int l = 0; l < 4; ++l) p->Bp[4 * j + l] = pair(d->t.B[8 * j + 2 * l], d->t.B[8 * j + 2 * l + 1]);
   }
   p->M = M; p->K = K; p->m_pad = static_cast<int>(AL.m_pad);
   p->kind = d->t.kind; p->center = d->center;
   p->katoms = sf_katoms(K);
-  // groups of R rows, one thread per 32-element block
-  int R = static_cast<int>(cdiv(256, nb));
-  const int r_mem = static_cast<int>(32768 / (static_cast<size_t>(K) * 2));
-  if (R > r_mem) R = r_mem;
-  if (R > 64) R = 64;
-  if (R < 1) R = 1;
-  const int items = R * nb;
+  // groups of R rows; each row staged in a 512-byte aligned slot (its own 64-byte
+  // swizzle pattern), loaded in boxes of up to 256 lines. Centring: each of the 4
+  // consumer warps owns U whole rows; otherwise the consumers stride over the blocks.
+  const uint32_t rstride = static_cast<uint32_t>(align_up(static_cast<size_t>(K) * 2, 512));
+  const int nwc = 4;
+  int U = 1, R = 1;
+  if (d->center) {
+    U = static_cast<int>((64 + nb / 2) / nb);
+    if (U < 1) U = 1;
+    if (U > 16) U = 16;
+    R = nwc * U;
+  } else {
+    R = static_cast<int>((4 * 128 + nb / 2) / nb);
+    if (R < 1) R = 1;
+    if (R > 64) R = 64;
+  }
+  while (R > 1 && static_cast<size_t>(R) * rstride > 96 * 1024) {   // keep a slot <= 96 KB
+    if (d->center) { if (U == 1) break; --U; R = nwc * U; } else { --R; }
+  }
   int box = 1;
-  for (int c = 1; c <= 256 && c <= items; ++c) if (items % c == 0) box = c;
+  for (int c = 1; c <= 256 && c <= nb; ++c) if (nb % c == 0) box = c;
   p->rows_per_group = R;
+  p->rows_per_warp = U;
+  p->consumer_warps = nwc;
   p->box_lines = box;
+  p->row_stride = rstride;
   if (!make_tmap(&p->tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, 32,
                  static_cast<uint64_t>(M) * nb, 64, 32, static_cast<uint32_t>(box),
                  CU_TENSOR_MAP_SWIZZLE_64B))
     return KQ_ERR_CUDA;
-  const int nb_pad = static_cast<int>(p->katoms) * 4;
-  size_t off = 1024 + align_up(static_cast<size_t>(R) * nb_pad, 16) + static_cast<size_t>(items) * 4;
-  p->tables_off = align_up(off, 128);
-  const size_t tables = d->t.kind == KQ_T_RPBH ? static_cast<size_t>(K) * 2 + static_cast<size_t>(nb) * 4 : 0;
+  p->tables_off = 1024;
+  const size_t tables = d->t.kind == KQ_T_RPBH ? static_cast<size_t>(K) * 2 + static_cast<size_t>(nb) * 16 : 0;
   p->bufs_off = align_up(p->tables_off + tables, 1024);
-  const size_t buf_bytes = align_up(static_cast<size_t>(items) * 64, 1024);
-  const size_t budget = 227 * 1024;
+  const size_t buf_bytes = align_up(static_cast<size_t>(R) * rstride, 1024);
+  // prefer a footprint that lets two CTAs share an SM; fall back to the full budget
+  size_t budget = 113 * 1024;
+  if (p->bufs_off + 2 * buf_bytes > budget) budget = 227 * 1024;
   if (p->bufs_off + buf_bytes > budget) return KQ_ERR_UNSUPPORTED_SHAPE;
   p->nbufs = static_cast<int>((budget - p->bufs_off) / buf_bytes);
   if (p->nbufs > 4) p->nbufs = 4;
   p->smem_bytes = p->bufs_off + static_cast<size_t>(p->nbufs) * buf_bytes;
-  if (d->t.kind == KQ_T_RPBH && K > 65536) return KQ_ERR_UNSUPPORTED_SHAPE;
+  if (d->t.kind == KQ_T_RPBH && K * 2 > 65535) return KQ_ERR_UNSUPPORTED_SHAPE;
   (void)di;
   if (act) {
     p->codes = act + AL.codes;
@@ -225,8 +248,9 @@ kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* 
                    kUCols, static_cast<uint64_t>(d->K) * 2, 64, kUCols, CU_TENSOR_MAP_SWIZZLE_128B))
       return KQ_ERR_CUDA;
     lp.c1 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(weights) + WL.c1);
+    lp.mu = d->center ? reinterpret_cast<const float*>(act + AL.mu) : nullptr;
     lp.u = reinterpret_cast<uint16_t*>(act + AL.u);
-    lp.M = M; lp.K = d->K; lp.center = d->center;
+    lp.M = M; lp.K = d->K; lp.split = u_split(M, d->K);
     lp.err = reinterpret_cast<uint32_t*>(act + AL.err);
     if (launch_lowrank_u(lp, st) != cudaSuccess) return KQ_ERR_CUDA;
   }
@@ -252,10 +276,10 @@ kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* a
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return KQ_ERR_CUDA;
   if (d->rank > 0) {
-    if (!make_tmap(&gp.tmap_u, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, act + AL.u, kRankPad,
+    if (!make_tmap(&gp.tmap_u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act + AL.u, kRankPad,
                    static_cast<uint64_t>(M), kRankPad * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return KQ_ERR_CUDA;
-    if (!make_tmap(&gp.tmap_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w + WL.l2t, kRankPad,
+    if (!make_tmap(&gp.tmap_l2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w + WL.l2t, kRankPad,
                    static_cast<uint64_t>(N), kRankPad * 2, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))
       return KQ_ERR_CUDA;
   }
@@ -367,6 +391,7 @@ kq_status kq_quantize_act(const kq_layer_desc* desc, const void* weights, const 
   DeviceInfo di;
   if ((s = current_device(&di)) != KQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // the error word starts at zero for this call
   if (cudaMemsetAsync(act, 0, 4, st) != cudaSuccess) return KQ_ERR_CUDA;
   return run_quantize(desc, weights, X_bf16, M, static_cast<uint8_t*>(act), st, di);
 }

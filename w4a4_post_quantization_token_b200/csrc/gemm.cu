@@ -1,7 +1,7 @@
 // Contraction half of the W4A4 linear layer on the 5th-generation tensor cores:
 //
 //   Y[m, n] = sum_k deq(Xq)[m, k] deq(Rq)[n, k]          (tcgen05 kind::mxf4, block32)
-//           + sum_j U[m, j] L2t[n, j]                     (tcgen05 kind::f16, same accumulator)
+//           + sum_j U[m, j] L2t[n, j]                     (tcgen05 kind::f16, fp16, same accumulator)
 //           + mu[m] s[n]                                  (fp32 epilogue)
 //
 // The first term is the 4-bit x 4-bit product the KroQuant commentary (sections 01, 03)
@@ -16,7 +16,7 @@
 //   warp 1     TMEM allocator and single-thread MMA issuer. Two TMEM accumulators
 //              (2 x 192 columns) alternate between tiles, so the epilogue of one tile
 //              overlaps the MMAs of the next. Per k-tile: tcgen05.cp of the scales into
-//              TMEM, then block-scaled MMAs (K = 64 each); per tile: 4 bf16 MMAs for the
+//              TMEM, then block-scaled MMAs (K = 64 each); per tile: 4 fp16 MMAs for the
 //              low-rank branch; tcgen05.commit frees ring slots / hands over accumulators.
 //   warps 2-5  epilogue: tcgen05.ld 32 columns at a time, + mu[m] s[n], convert, write a
 //              128-byte-swizzled staging tile in shared memory, TMA-store it (async).
@@ -172,7 +172,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_mxf4(const __grid_constant__ Ge
                        (ks > 0 || kk > 0) ? 1u : 0u);
             }
           } else {
-            constexpr uint32_t idesc = idesc_bf16(kBM, kBN);
+            constexpr uint32_t idesc = idesc_f16(kBM, kBN);      // U and L2^T are fp16
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk)
               mma_bf16(d, sdesc_sw128_kmajor(a + 32 * kk), sdesc_sw128_kmajor(b + 32 * kk), idesc,

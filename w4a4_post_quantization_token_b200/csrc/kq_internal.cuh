@@ -14,10 +14,11 @@ namespace kq {
 
 struct QuantParams {
   CUtensorMap tmap_x;          // X viewed as [M * K/32 lines, 32 bf16], 64-byte swizzle
-  float A[16];                 // Kronecker factor A (4x4, row-major)
-  float B[64];                 // Kronecker factor B (8x8, row-major)
+  uint64_t Ap[16];             // Kronecker A as pairs (A[i][k], A[i][k]), index 4 i + k
+  uint64_t Bp[32];             // Kronecker B as pairs (B[j][2l], B[j][2l+1]), index 4 j + l
   int M, K, m_pad, kind, center;
-  int rows_per_group, box_lines, nbufs;
+  int rows_per_group, rows_per_warp, consumer_warps, box_lines, nbufs;
+  uint32_t row_stride;         // bytes between staged rows (512-byte multiple)
   size_t tables_off, bufs_off, smem_bytes;   // dynamic shared memory carve-up
   int64_t katoms;
   uint8_t* codes;              // act codes [M, K/2]
@@ -33,16 +34,17 @@ struct LowRankParams {
   CUtensorMap tmap_x;          // X [M, K] bf16, box 64 x 128, 128-byte swizzle
   CUtensorMap tmap_l1;         // [kUCols, K] bf16, box 64 x kUCols, 128-byte swizzle
   const float* c1;             // [64]
-  uint16_t* u;                 // U [M, 64] bf16
-  int M, K, center;
+  const float* mu;             // [M] token means (null without centring)
+  uint16_t* u;                 // U [M, 64] fp16
+  int M, K, split;             // split: CTAs (one cluster) per 128-row tile, 1/2/4/8
   uint32_t* err;
 };
 
 struct GemmParams {
   CUtensorMap tmap_a;          // act codes [M, K/2] uint8, box 128 x 128, 128-byte swizzle
   CUtensorMap tmap_b;          // residual codes [N, K/2] uint8, box 128 x BN
-  CUtensorMap tmap_u;          // U [M, 64] bf16, box 64 x 128
-  CUtensorMap tmap_l2;         // L2^T [N, 64] bf16, box 64 x BN
+  CUtensorMap tmap_u;          // U [M, 64] fp16, box 64 x 128
+  CUtensorMap tmap_l2;         // L2^T [N, 64] fp16, box 64 x BN
   CUtensorMap tmap_y;          // Y [M, N] f32 or bf16, box (128 bytes) x 32 rows, 128-byte swizzle
   const uint8_t* sfa;          // act scales (tensor-core layout)
   const uint8_t* sfb;          // residual scales (tensor-core layout, one spare row atom)

@@ -16,7 +16,9 @@ namespace kq {
 constexpr int kBlock = 32;          // MXFP4 block size along K
 constexpr int kTileK = 256;         // FP4 elements per GEMM k-tile (128 bytes per row)
 constexpr int kRankPad = 64;        // low-rank dimension as stored (rank <= 64)
-constexpr int kUCols = 2 * kRankPad + 16;   // U-kernel MMA width: L1' hi, L1' lo, ones row
+constexpr int kUCols = 2 * kRankPad;         // U-kernel MMA width: L1' hi, L1' lo
+constexpr int kUSplitMax = 8;                // largest split of K in the U kernel
+constexpr int kHdrBytes = 256;               // workspace header: the device error word
 constexpr size_t kAlign = 1024;
 
 __host__ __device__ constexpr size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -39,8 +41,8 @@ struct WeightsLayout {
   int kind = 0;
   size_t rcodes = 0;   // uint8 [N, K/2]     residual codes (R^T, K-major)
   size_t rsf = 0;      // uint8 tiled        residual scales, rows padded (see n_pad)
-  size_t l2t = 0;      // bf16  [N, rp]      L2^T (K-major B operand of the low-rank MMA)
-  size_t l1t = 0;      // bf16  [kUCols, K]  rows 0..63 L1'^T hi, 64..127 lo, 128 ones
+  size_t l2t = 0;      // fp16  [N, rp]      L2^T (K-major B operand of the low-rank MMA)
+  size_t l1t = 0;      // bf16  [kUCols, K]  rows 0..63 L1'^T hi, 64..127 lo
   size_t c1 = 0;       // f32   [rp]         1^T (L1' hi + lo)
   size_t s = 0;        // f32   [N]          1^T W
   size_t perm = 0;     // int32 [K]          RPBH gather indices
@@ -69,13 +71,22 @@ struct WeightsLayout {
   }
 };
 
+// Split of the K reduction in the U kernel (a power of two <= 8): enough CTAs for a full
+// GPU when M is small. The splits of one 128-row tile form a thread-block cluster.
+__host__ __device__ constexpr int u_split(int64_t M, int64_t K) {
+  const int64_t mt = cdiv(M, 128), kt = cdiv(K, 64);
+  int s = 1;
+  while (s < kUSplitMax && mt * (2 * s) <= 148 && 2 * (2 * s) <= kt) s *= 2;
+  return s;
+}
+
 struct ActLayout {
   int64_t M = 0, m_pad = 0, K = 0, rp = 0;
   size_t err = 0;      // uint32 device error word
   size_t codes = 0;    // uint8 [M, K/2]
   size_t sf = 0;       // uint8 tiled, rows padded to 128
   size_t mu = 0;       // f32 [m_pad]
-  size_t u = 0;        // bf16 [M, rp]
+  size_t u = 0;        // fp16 [M, rp]
   size_t total = 0;
 
   __host__ __device__ static ActLayout make(int64_t M, int64_t K, int64_t rank) {
@@ -83,7 +94,7 @@ struct ActLayout {
     L.M = M; L.K = K; L.rp = rank > 0 ? kRankPad : 0;
     L.m_pad = cdiv(M, 128) * 128;
     size_t o = 0;
-    L.err = o;    o = 256;
+    L.err = o;    o = kHdrBytes;
     L.codes = o;  o = align_up(o + static_cast<size_t>(M) * (K / 2), kAlign);
     L.sf = o;     o = align_up(o + sf_bytes(L.m_pad, K), kAlign);
     L.mu = o;     o = align_up(o + static_cast<size_t>(L.m_pad) * 4, kAlign);

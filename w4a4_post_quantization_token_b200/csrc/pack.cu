@@ -2,6 +2,7 @@
 // [rows, K/32], low-rank factors) and the internal tensor-core layouts of the
 // prepared-weights buffer and the activation workspace.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kq_pack.cuh"
 
@@ -46,20 +47,30 @@ __global__ void k_unpad_cols_bf16(const uint16_t* __restrict__ src, int64_t rows
   dst[t] = src[r * kRankPad + j];
 }
 
-// L2 [r, N] bf16 -> l2t [N, 64]
+// L2 [r, N] bf16 -> l2t [N, 64] fp16 (exact for |L2| in [2^-14, 65504])
 __global__ void k_l2_to_l2t(const uint16_t* __restrict__ L2, int r, int N, uint16_t* __restrict__ l2t) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= static_cast<int64_t>(N) * kRankPad) return;
   const int n = static_cast<int>(t / kRankPad);
   const int j = static_cast<int>(t % kRankPad);
-  l2t[t] = j < r ? L2[static_cast<int64_t>(j) * N + n] : static_cast<uint16_t>(0);
+  uint16_t out = 0;
+  if (j < r) {
+    const float v = __uint_as_float(static_cast<uint32_t>(L2[static_cast<int64_t>(j) * N + n]) << 16);
+    const __half h = __float2half_rn(v);
+    out = *reinterpret_cast<const uint16_t*>(&h);
+  }
+  l2t[t] = out;
 }
+// l2t fp16 -> L2 [r, N] bf16
 __global__ void k_l2t_to_l2(const uint16_t* __restrict__ l2t, int r, int N, uint16_t* __restrict__ L2) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= static_cast<int64_t>(r) * N) return;
   const int j = static_cast<int>(t / N);
   const int n = static_cast<int>(t % N);
-  L2[t] = l2t[static_cast<int64_t>(n) * kRankPad + j];
+  const uint16_t hb = l2t[static_cast<int64_t>(n) * kRankPad + j];
+  const float v = __half2float(*reinterpret_cast<const __half*>(&hb));
+  const __nv_bfloat16 b = __float2bfloat16_rn(v);
+  L2[t] = *reinterpret_cast<const uint16_t*>(&b);
 }
 
 __device__ __forceinline__ uint16_t f32_to_bf16_bits_rn(float x) {
@@ -67,7 +78,7 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits_rn(float x) {
   return *reinterpret_cast<const uint16_t*>(&h);
 }
 
-// L1' float32 [K, r] -> l1t rows: t = hi, 64 + t = lo (bf16), row 128 = ones
+// L1' float32 [K, r] -> l1t rows: t = hi, 64 + t = lo (bf16)
 __global__ void k_l1p_to_l1t(const float* __restrict__ L1p, int K, int r, uint16_t* __restrict__ l1t) {
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= static_cast<int64_t>(K) * kRankPad) return;
@@ -81,7 +92,6 @@ __global__ void k_l1p_to_l1t(const float* __restrict__ L1p, int K, int r, uint16
   }
   l1t[static_cast<int64_t>(j) * K + k] = hi;
   l1t[static_cast<int64_t>(kRankPad + j) * K + k] = lo;
-  if (j == 0) l1t[static_cast<int64_t>(2 * kRankPad) * K + k] = 0x3F80u;
 }
 
 // c1[j] = sum_k (hi + lo)   (fp64 accumulate), one block per j < 64

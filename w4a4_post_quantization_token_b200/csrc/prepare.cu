@@ -12,6 +12,7 @@
 #include <cublas_v2.h>
 #include <cusolverDn.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include <cmath>
 #include <vector>
@@ -194,18 +195,14 @@ __global__ void k_rowsum_f64(const double* __restrict__ L1p, int K, float* __res
   if (threadIdx.x == 0) c1[t] = static_cast<float>(red[0]);
 }
 
-// l2t[n][t] = bf16(L2bT[n + t N]) for t < r
+// l2t[n][t] = fp16 of the bf16-rounded L2[t][n] (exact for |L2| in [2^-14, 65504]) for t < r
 __global__ void k_store_l2t(const double* __restrict__ L2bT, int N, int r, uint16_t* __restrict__ l2t) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
-  for (int t = 0; t < r; ++t)
-    l2t[static_cast<size_t>(n) * kRankPad + t] = f64_to_bf16_bits(L2bT[static_cast<size_t>(t) * N + n]);
-}
-
-// ones row (index 2 * kRankPad) of l1t
-__global__ void k_fill_ones(uint16_t* __restrict__ row, int K) {
-  const int k = blockIdx.x * blockDim.x + threadIdx.x;
-  if (k < K) row[k] = 0x3F80u;   // bf16 1.0
+  for (int t = 0; t < r; ++t) {
+    const __half h = __double2half(L2bT[static_cast<size_t>(t) * N + n]);
+    l2t[static_cast<size_t>(n) * kRankPad + t] = *reinterpret_cast<const uint16_t*>(&h);
+  }
 }
 
 // ------------------------------------------------------------------------------------
@@ -315,8 +312,6 @@ PrepStatus run_prepare(const PrepareArgs& a) {
       k_rowsum_f64<<<r, 256, 0, st>>>(L1p, K, reinterpret_cast<float*>(w + WL.c1));
       k_store_l2t<<<static_cast<unsigned>(cdiv(N, 256)), 256, 0, st>>>(L2bT, N, r,
                                                                         reinterpret_cast<uint16_t*>(w + WL.l2t));
-      k_fill_ones<<<static_cast<unsigned>(cdiv(K, 256)), 256, 0, st>>>(
-          reinterpret_cast<uint16_t*>(w + WL.l1t) + static_cast<size_t>(2 * kRankPad) * K, K);
       if (cudaGetLastError() != cudaSuccess) { status = PrepStatus::Cuda; break; }
     } while (false);
     if (status == PrepStatus::Ok) {

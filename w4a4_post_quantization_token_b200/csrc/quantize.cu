@@ -12,11 +12,14 @@
 //    RPBH(X) = X P H D). MXFP4 encoding as in encode.cuh (KroQuant section 03).
 //  * k_lowrank_u -- U = X L1' - mu c1 (SVDQuant explainer, section 3: the low-rank branch
 //    runs on the high-precision input) as a tcgen05 bf16 GEMM: TMA loads 128x64 tiles of
-//    X and of [L1'_hi; L1'_lo; 1], the MMA accumulates 128 x 144 in TMEM, the epilogue
-//    forms hi + lo - (rowsum / K) c1 and stores bf16.
+//    X and of [L1'_hi; L1'_lo], the MMA accumulates 128 x 128 in TMEM, the epilogue forms
+//    hi + lo - mu c1 (mu from the quantize kernel) and stores fp16 (16-bit branch). For
+//    small M the K reduction is split over a cluster and reduced in distributed smem.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "kq_internal.cuh"
+#include "packed.cuh"
 
 namespace kq {
 
@@ -69,224 +72,325 @@ __device__ __forceinline__ double warp_sum_f64(double x) {
   return x;
 }
 
-// x (A (x) B) for one block: X_m[i][j] = v[8 i + j], out = A^T X_m B.
-__device__ __forceinline__ void kron_apply(float (&v)[32], const float* __restrict__ A,
-                                           const float* __restrict__ B) {
-  float t[32];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int l = 0; l < 8; ++l) {
-      float acc = v[8 * i] * B[l];
-#pragma unroll
-      for (int j = 1; j < 8; ++j) acc = fmaf(v[8 * i + j], B[8 * j + l], acc);
-      t[8 * i + l] = acc;
-    }
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-#pragma unroll
-    for (int l = 0; l < 8; ++l) {
-      float acc = A[k] * t[l];
-#pragma unroll
-      for (int i = 1; i < 4; ++i) acc = fmaf(A[4 * i + k], t[8 * i + l], acc);
-      v[8 * k + l] = acc;
-    }
-}
-
-// In-place 32-point Walsh-Hadamard transform in Sylvester order (unnormalised).
-__device__ __forceinline__ void fwht32(float (&v)[32]) {
-#pragma unroll
-  for (int h = 1; h < 32; h <<= 1)
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if ((i & h) == 0) {
-        const float a = v[i], b = v[i + h];
-        v[i] = a + b;
-        v[i + h] = a - b;
-      }
-}
-
 // ----------------------------------------------------------------------------------
 // k_quantize_rows
 // ----------------------------------------------------------------------------------
-// One CTA processes groups of R consecutive token rows; one thread per 32-element block
-// (R * K/32 threads). Groups are staged by TMA (64-byte swizzle, one 64-byte line per
-// block) into a ring of up to 4 slots; the CTA walks groups blockIdx.x, +gridDim.x, ...
+// Groups of R consecutive token rows; each row is staged by TMA (64-byte swizzle, one
+// 64-byte line per 32-element block) into its own 512-byte aligned slot of a ring of up
+// to 4 group buffers; one consumer lane per block. The CTA walks groups blockIdx.x,
+// +gridDim.x, ... Arithmetic runs on fp32 pairs (Blackwell f32x2 FMA/ADD/SUB/MUL), each
+// lane rounded like the scalar instruction.
+
+// Kronecker apply on pairs: v2[4i + jp] = (x[8i+2jp], x[8i+2jp+1]);
+// T[i][l] = sum_j x[8i+j] B[j][l] with Bp[4j + lp] = (B[j][2lp], B[j][2lp+1]);
+// Y[k][l] = sum_i A[i][k] T[i][l] with Ap[4i + k] = (A[i][k], A[i][k]).
+__device__ __forceinline__ void kron_apply2(uint64_t (&v2)[16], const uint64_t* __restrict__ Ap,
+                                            const uint64_t* __restrict__ Bp) {
+  uint64_t t2[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint64_t acc[4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float x = (j & 1) ? f2hi(v2[4 * i + j / 2]) : f2lo(v2[4 * i + j / 2]);
+      const uint64_t xx = f2pack(x, x);
+#pragma unroll
+      for (int lp = 0; lp < 4; ++lp)
+        acc[lp] = j == 0 ? fmul2(xx, Bp[lp]) : ffma2(xx, Bp[4 * j + lp], acc[lp]);
+    }
+#pragma unroll
+    for (int lp = 0; lp < 4; ++lp) t2[4 * i + lp] = acc[lp];
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int lp = 0; lp < 4; ++lp) {
+      uint64_t acc = fmul2(Ap[k], t2[lp]);
+#pragma unroll
+      for (int i = 1; i < 4; ++i) acc = ffma2(Ap[4 * i + k], t2[4 * i + lp], acc);
+      v2[4 * k + lp] = acc;
+    }
+}
+
+// Unnormalised 32-point Walsh-Hadamard transform (Sylvester order) on pairs.
+__device__ __forceinline__ void fwht32_2(uint64_t (&v2)[16]) {
+#pragma unroll
+  for (int hp = 1; hp < 16; hp <<= 1)          // element strides 2, 4, 8, 16
+#pragma unroll
+    for (int p = 0; p < 16; ++p)
+      if ((p & hp) == 0) {
+        const uint64_t a = v2[p], b = v2[p + hp];
+        v2[p] = fadd2(a, b);
+        v2[p + hp] = fsub2(a, b);
+      }
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {                // element stride 1: inside each pair
+    float a, b;
+    f2unpack(v2[p], a, b);
+    v2[p] = f2pack(a + b, a - b);
+  }
+}
+
+__device__ __forceinline__ float amax32_2(const uint64_t (&v2)[16]) {
+  float m = 0.f;
+#pragma unroll
+  for (int p = 0; p < 16; ++p) {
+    float a, b;
+    f2unpack(v2[p], a, b);
+    m = fmaxf(m, fmaxf(fabsf(a), fabsf(b)));
+  }
+  return m;
+}
+
+// codes of v2 * f (f a scale whose product with each value is the value / 2^e)
+__device__ __forceinline__ void encode_scaled2(const uint64_t (&v2)[16], float f, uint32_t (&c)[4]) {
+  const uint64_t ff = f2pack(f, f);
+#pragma unroll
+  for (int w = 0; w < 4; ++w)
+    c[w] = cvt_e2m1x8(fmul2(v2[4 * w], ff), fmul2(v2[4 * w + 1], ff), fmul2(v2[4 * w + 2], ff),
+                      fmul2(v2[4 * w + 3], ff));
+}
+
 constexpr int kQMaxBufs = 4;
 
+// Transform + encode of one 32-element block (row r of the ring slot, block b). Writes the
+// codes (or, in debug mode, the transformed values) and returns the scale byte.
+template <int KIND, bool CENTER, bool DEBUG_XT>
+__device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const uint8_t* rowb,
+                                                   const uint8_t* tables, int row, int b,
+                                                   float mu_hi, float mu_lo) {
+  const float rs = 0.17677669529663687f;   // fp32(1 / sqrt(32))
+  uint64_t v2[16];
+  if (KIND == 2) {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 ix = *reinterpret_cast<const uint4*>(
+          tables + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
+      const uint32_t w4[4] = {ix.x, ix.y, ix.z, ix.w};
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const uint16_t h0 = *reinterpret_cast<const uint16_t*>(rowb + (w4[t] & 0xFFFFu));
+        const uint16_t h1 = *reinterpret_cast<const uint16_t*>(rowb + (w4[t] >> 16));
+        v2[4 * c + t] = f2pack(__uint_as_float(static_cast<uint32_t>(h0) << 16),
+                               __uint_as_float(static_cast<uint32_t>(h1) << 16));
+      }
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 q = *reinterpret_cast<const uint4*>(rowb + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
+      v2[4 * c + 0] = bf16x2_to_f2(q.x);
+      v2[4 * c + 1] = bf16x2_to_f2(q.y);
+      v2[4 * c + 2] = bf16x2_to_f2(q.z);
+      v2[4 * c + 3] = bf16x2_to_f2(q.w);
+    }
+  }
+  if (CENTER) {
+    const uint64_t mh = f2pack(mu_hi, mu_hi), ml = f2pack(mu_lo, mu_lo);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) v2[q] = fsub2(fsub2(v2[q], mh), ml);
+  }
+  if (KIND == 1) kron_apply2(v2, p.Ap, p.Bp);
+  if (KIND == 2) fwht32_2(v2);
+  const uint32_t* signs = reinterpret_cast<const uint32_t*>(tables + static_cast<size_t>(p.K) * 2);
+  if (DEBUG_XT) {
+    if (KIND == 2) {
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        float a, c2;
+        f2unpack(v2[q], a, c2);
+        const uint32_t mw = signs[4 * b + q / 4];
+        const uint32_t s0 = (mw >> (4 * (2 * (q % 4)) + 3)) & 1u;
+        const uint32_t s1 = (mw >> (4 * (2 * (q % 4) + 1) + 3)) & 1u;
+        v2[q] = f2pack(__uint_as_float(__float_as_uint(a * rs) ^ (s0 << 31)),
+                       __uint_as_float(__float_as_uint(c2 * rs) ^ (s1 << 31)));
+      }
+    }
+    float4* o = reinterpret_cast<float4*>(p.xt + static_cast<size_t>(row) * p.K + b * kBlock);
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      o[q] = make_float4(f2lo(v2[2 * q]), f2hi(v2[2 * q]), f2lo(v2[2 * q + 1]), f2hi(v2[2 * q + 1]));
+    return 0u;
+  }
+  uint32_t c[4];
+  uint32_t sbyte;
+  if (KIND == 2) {
+    // Xt = y * rs * sign. amax(y * rs) = fl(amax(y) * rs) (rounding is monotonic), and
+    // fl(y * rs) / 2^e = fl(y * (rs / 2^e)) (power-of-two scaling commutes with rounding
+    // for normal results); the sign flips the code's sign bit.
+    sbyte = mx_scale_byte(amax32_2(v2) * rs);
+    if (sbyte > 0) {
+      encode_scaled2(v2, rs * mx_inv_scale(sbyte), c);
+    } else {
+      const uint64_t rr = f2pack(rs, rs);       // tiny block: keep the two-step rounding
+#pragma unroll
+      for (int q = 0; q < 16; ++q) v2[q] = fmul2(v2[q], rr);
+      encode_scaled2(v2, mx_inv_scale(sbyte), c);
+    }
+    const uint4 sg = *reinterpret_cast<const uint4*>(signs + 4 * b);
+    c[0] ^= sg.x; c[1] ^= sg.y; c[2] ^= sg.z; c[3] ^= sg.w;
+  } else {
+    sbyte = mx_scale_byte(amax32_2(v2));
+    encode_scaled2(v2, mx_inv_scale(sbyte), c);
+  }
+  *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + b * 16) =
+      make_uint4(c[0], c[1], c[2], c[3]);
+  return sbyte;
+}
+
+// Scale bytes of 4 consecutive blocks held by 4 consecutive lanes (lane % 4 == 0 is the
+// first) become one 32-bit word; or, when K/32 is not a multiple of 4, single bytes.
+__device__ __forceinline__ void store_scales(const QuantParams& p, bool valid, int row, int b,
+                                             int nb, int nb_pad, uint32_t sbyte) {
+  const int lane = threadIdx.x & 31;
+  if ((nb & 3) == 0) {
+    const uint32_t w = sbyte | (__shfl_down_sync(0xffffffffu, sbyte, 1) << 8) |
+                       (__shfl_down_sync(0xffffffffu, sbyte, 2) << 16) |
+                       (__shfl_down_sync(0xffffffffu, sbyte, 3) << 24);
+    if (valid && (lane & 3) == 0) {
+      *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, b, p.katoms)) = w;
+      if (b + 4 == nb)                                   // zero the padding blocks of the row
+        for (int bb = nb; bb < nb_pad; bb += 4)
+          *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, bb, p.katoms)) = 0u;
+    }
+  } else if (valid) {
+    p.sf[sf_offset(row, b, p.katoms)] = static_cast<uint8_t>(sbyte);
+    if (b == nb - 1)
+      for (int bb = nb; bb < nb_pad; ++bb) p.sf[sf_offset(row, bb, p.katoms)] = 0;
+  }
+}
+
+// Warp-specialised: warp NWc (the last) issues TMA loads of R-row groups into a ring of
+// S slots (one 512-byte aligned slot per row); warps 0..NWc-1 consume. A slot is handed
+// back through an mbarrier that every consumer warp arrives on. Centring: each consumer
+// warp owns U whole rows of the group, so a token's mean is a warp-local reduction.
+// Without centring the consumers stride over all blocks of the group.
 template <int KIND, bool CENTER, bool DEBUG_XT>
 __global__ void __launch_bounds__(512, 1) k_quantize_rows(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int NWc = static_cast<int>(blockDim.x >> 5) - 1;          // consumer warps
   const int nb = p.K / kBlock;
   const int nb_pad = static_cast<int>(p.katoms) * 4;
   const int R = p.rows_per_group;
+  const int U = p.rows_per_warp;                                   // centring only
   const int items = R * nb;
-  const uint32_t grp_bytes = static_cast<uint32_t>(items) * 64u;
-  const uint32_t buf_bytes = static_cast<uint32_t>(align_up(grp_bytes, 1024));
-  // shared memory carve-up
-  const int nbufs = p.nbufs;                                                 // <= kQMaxBufs
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);                       // [nbufs]
-  float2* mus = reinterpret_cast<float2*>(smem + 64);                       // [R] (hi, lo)
-  uint8_t* sst = smem + 64 + 8 * 64;                                        // scale staging
-  float* bsum = reinterpret_cast<float*>(smem + 1024 + align_up(static_cast<size_t>(R) * nb_pad, 16));
-  uint8_t* tables = smem + p.tables_off;                                    // RPBH tables
+  const uint32_t rstride = p.row_stride;
+  const uint32_t buf_bytes = static_cast<uint32_t>(align_up(static_cast<size_t>(R) * rstride, 1024));
+  const int S = p.nbufs;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);             // [S]
+  uint64_t* empty = full + kQMaxBufs;                              // [S]
+  uint8_t* tables = smem + p.tables_off;
   uint8_t* bufs = smem + p.bufs_off;
-
   const int ngroups = static_cast<int>(cdiv(p.M, R));
+
   if (tid == 0) {
-    for (int b = 0; b < nbufs; ++b) mbar_init(&full[b], 1);
+    for (int b = 0; b < S; ++b) { mbar_init(&full[b], 1); mbar_init(&empty[b], NWc); }
     fence_mbar_init();
     prefetch_tmap(&p.tmap_x);
   }
   if (KIND == 2) {
-    // perm as uint16, block b's 32 entries (64 bytes) with 16-byte chunks swizzled like the rows;
-    // sign bits: one 32-bit word per block
     uint16_t* pt = reinterpret_cast<uint16_t*>(tables);
-    uint32_t* sb = reinterpret_cast<uint32_t*>(tables + static_cast<size_t>(p.K) * 2);
-    for (int k = tid; k < p.K; k += blockDim.x) {
-      const uint32_t off = static_cast<uint32_t>(k) * 2u;
-      pt[swz64(off) / 2] = static_cast<uint16_t>(p.perm[k]);
-    }
-    for (int b = tid; b < nb; b += blockDim.x) {
-      uint32_t w = 0;
-      for (int j = 0; j < 32; ++j) w |= (p.sgn[32 * b + j] < 0.f ? 1u : 0u) << j;
-      sb[b] = w;
-    }
+    uint32_t* sm = reinterpret_cast<uint32_t*>(tables + static_cast<size_t>(p.K) * 2);
+    for (int k = tid; k < p.K; k += blockDim.x)
+      pt[swz64(static_cast<uint32_t>(k) * 2u) / 2] =
+          static_cast<uint16_t>(swz64(static_cast<uint32_t>(p.perm[k]) * 2u));
+    for (int b = tid; b < nb; b += blockDim.x)
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        uint32_t m = 0;
+        for (int j = 0; j < 8; ++j) m |= (p.sgn[32 * b + 8 * w + j] < 0.f ? 8u : 0u) << (4 * j);
+        sm[4 * b + w] = m;
+      }
   }
   __syncthreads();
 
-  auto issue = [&](int g, int buf) {
-    uint8_t* dst = bufs + static_cast<size_t>(buf) * buf_bytes;
-    mbar_arrive_expect_tx(&full[buf], grp_bytes);
-    const int l0 = g * items;
-    for (int l = 0; l < items; l += p.box_lines)
-      tma_load_2d(dst + static_cast<size_t>(l) * 64u, &p.tmap_x, 0, l0 + l, &full[buf]);
-  };
-  if (tid == 0)
-    for (int b = 0; b < nbufs; ++b) {
-      const int g = blockIdx.x + b * gridDim.x;
-      if (g < ngroups) issue(g, b);
-    }
-
-  int iter = 0;
-  for (int g = blockIdx.x; g < ngroups; g += gridDim.x, ++iter) {
-    const int buf = iter % nbufs;
-    const uint32_t parity = static_cast<uint32_t>(iter / nbufs) & 1u;
-    const int row0 = g * R;
-    __syncthreads();   // previous group's staging reads are done
-    const bool ok = __syncthreads_and(mbar_wait(&full[buf], parity, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
-    if (!ok) break;
-    const uint8_t* gbuf = bufs + static_cast<size_t>(buf) * buf_bytes;
-
-    if (CENTER) {
-      for (int i = tid; i < items; i += blockDim.x) {
-        float v[32];
-        load_block_swz(gbuf, i, v);
-        bsum[i] = tree_sum32(v);
+  if (warp == NWc) {
+    // ----------------------------------------------------------------- producer
+    if (lane == 0) {
+      int k = 0;
+      for (int g = blockIdx.x; g < ngroups; g += gridDim.x, ++k) {
+        const int s = k % S;
+        if (k >= S && !mbar_wait(&empty[s], ((k / S) - 1) & 1, p.err, KQ_DEV_ERR_TIMEOUT_EMPTY)) break;
+        uint8_t* dst = bufs + static_cast<size_t>(s) * buf_bytes;
+        const int rows = min(R, p.M - g * R);
+        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(rows) * nb * 64u);
+        for (int r = 0; r < rows; ++r)
+          for (int l = 0; l < nb; l += p.box_lines)
+            tma_load_2d(dst + static_cast<size_t>(r) * rstride + static_cast<size_t>(l) * 64u,
+                        &p.tmap_x, 0, (g * R + r) * nb + l, &full[s]);
       }
-      __syncthreads();
-      const int warp = tid >> 5, lane = tid & 31, nwarps = blockDim.x >> 5;
-      for (int r = warp; r < R; r += nwarps) {
-        double part = 0.0;
-        for (int b = lane; b < nb; b += 32) part += static_cast<double>(bsum[r * nb + b]);
-        const double mu64 = warp_sum_f64(part) / static_cast<double>(p.K);
-        const float hi = static_cast<float>(mu64);
-        const float lo = static_cast<float>(mu64 - static_cast<double>(hi));
-        if (lane == 0) {
-          mus[r] = make_float2(hi, lo);
-          if (row0 + r < p.M) p.mu[row0 + r] = hi;
-        }
-      }
-      __syncthreads();
-    } else if (tid < R && row0 + tid < p.M) {
-      p.mu[row0 + tid] = 0.f;
     }
-
-    for (int i = tid; i < items; i += blockDim.x) {
-      const int r = i / nb, b = i - r * nb;
-      const int row = row0 + r;
-      if (row >= p.M) continue;
-      float v[32];
-      // swizzle positions are taken relative to the 1024-byte aligned ring slot: line index
-      // i = r * nb + b for the block, element index r * K + e for a gathered element
-      if (KIND == 2) {
+  } else {
+    // ----------------------------------------------------------------- consumers
+    int k = 0;
+    for (int g = blockIdx.x; g < ngroups; g += gridDim.x, ++k) {
+      const int s = k % S;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / S) & 1, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
+      if (!ok) break;
+      const uint8_t* gbuf = bufs + static_cast<size_t>(s) * buf_bytes;
+      const int row0 = g * R;
+      if (CENTER) {
+        for (int u = 0; u < U; ++u) {
+          const int r = warp * U + u;
+          const int row = row0 + r;
+          if (row >= p.M) break;                                   // warp-uniform
+          const uint8_t* rowb = gbuf + static_cast<size_t>(r) * rstride;
+          double part = 0.0;
+          for (int b = lane; b < nb; b += 32) {
+            uint64_t acc = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 ix = *reinterpret_cast<const uint4*>(
-              tables + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
-          const uint32_t w4[4] = {ix.x, ix.y, ix.z, ix.w};
-#pragma unroll
-          for (int t = 0; t < 4; ++t) {
-            v[8 * c + 2 * t] = load_elem_swz(gbuf, r * p.K + static_cast<int>(w4[t] & 0xFFFFu));
-            v[8 * c + 2 * t + 1] = load_elem_swz(gbuf, r * p.K + static_cast<int>(w4[t] >> 16));
+            for (int c = 0; c < 4; ++c) {
+              const uint4 q = *reinterpret_cast<const uint4*>(rowb + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
+              const uint64_t s0 = fadd2(bf16x2_to_f2(q.x), bf16x2_to_f2(q.y));
+              const uint64_t s1 = fadd2(bf16x2_to_f2(q.z), bf16x2_to_f2(q.w));
+              acc = c == 0 ? fadd2(s0, s1) : fadd2(acc, fadd2(s0, s1));
+            }
+            part += static_cast<double>(f2lo(acc) + f2hi(acc));
+          }
+          const double mu64 = warp_sum_f64(part) / static_cast<double>(p.K);
+          const float mu_hi = static_cast<float>(mu64);
+          const float mu_lo = static_cast<float>(mu64 - static_cast<double>(mu_hi));
+          if (lane == 0) p.mu[row] = mu_hi;
+          const int iters = (nb + 31) / 32;
+          for (int t = 0; t < iters; ++t) {
+            const int b = 32 * t + lane;
+            const bool valid = b < nb;
+            uint32_t sb = 0;
+            if (valid) sb = quantize_block<KIND, CENTER, DEBUG_XT>(p, rowb, tables, row, b, mu_hi, mu_lo);
+            if (!DEBUG_XT) store_scales(p, valid, row, b, nb, nb_pad, sb);
           }
         }
       } else {
-        load_block_swz(gbuf, i, v);
-      }
-      if (CENTER) {
-        const float2 m = mus[r];
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] = (v[j] - m.x) - m.y;
-      }
-      if (KIND == 1) {
-        kron_apply(v, p.A, p.B);
-      } else if (KIND == 2) {
-        fwht32(v);
-        const uint32_t sbits = reinterpret_cast<const uint32_t*>(tables + static_cast<size_t>(p.K) * 2)[b];
-        const float rs = 0.17677669529663687f;   // 1 / sqrt(32)
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
-          v[j] = __uint_as_float(__float_as_uint(v[j] * rs) ^ (((sbits >> j) & 1u) << 31));
-      }
-      if (DEBUG_XT) {
-        float4* o = reinterpret_cast<float4*>(p.xt + static_cast<size_t>(row) * p.K + b * kBlock);
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-      } else {
-        uint32_t c[4];
-        const uint32_t sbyte = mx_encode32(v, c);
-        *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + b * 16) =
-            make_uint4(c[0], c[1], c[2], c[3]);
-        sst[r * nb_pad + b] = static_cast<uint8_t>(sbyte);
-      }
-    }
-    __syncthreads();   // all reads of this ring slot and all staged scales are done
-    if (tid == 0) {
-      const int gn = g + nbufs * gridDim.x;
-      if (gn < ngroups) {
-        fence_async_smem();
-        issue(gn, buf);
-      }
-    }
-    if (!DEBUG_XT) {
-      // scale words: 4 consecutive blocks of one row per 32-bit word, padding blocks = 0
-      const int wpr = nb_pad / 4;
-      for (int i = tid; i < R * wpr; i += blockDim.x) {
-        const int r = i / wpr, w = i - r * wpr;
-        const int row = row0 + r;
-        if (row >= p.M) continue;
-        uint32_t word = 0;
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int b = 4 * w + t;
-          const uint32_t v = b < nb ? sst[r * nb_pad + b] : 0u;
-          word |= v << (8 * t);
+        for (int r = warp * 32 + lane; r < R; r += NWc * 32)
+          if (row0 + r < p.M) p.mu[row0 + r] = 0.f;
+        const int span = NWc * 32;
+        const int iters = (items + span - 1) / span;
+        for (int t = 0; t < iters; ++t) {
+          const int i = t * span + warp * 32 + lane;
+          const int r = i / nb, b = i - r * nb;
+          const int row = row0 + r;
+          const bool valid = i < items && row < p.M;
+          uint32_t sb = 0;
+          if (valid)
+            sb = quantize_block<KIND, CENTER, DEBUG_XT>(p, gbuf + static_cast<size_t>(r) * rstride, tables,
+                                                         row, b, 0.f, 0.f);
+          if (!DEBUG_XT) store_scales(p, valid, row, b, nb, nb_pad, sb);
         }
-        *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, 4 * w, p.katoms)) = word;
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
     }
-  }
-  // rows M .. m_pad-1 of the last 128-row group: zero scales (finite values for the GEMM)
-  if (!DEBUG_XT) {
-    const int wpr = nb_pad / 4;
-    const int pad_rows = p.m_pad - p.M;
-    for (int i = blockIdx.x * blockDim.x + tid; i < pad_rows * wpr; i += gridDim.x * blockDim.x) {
-      const int r = p.M + i / wpr, w = i % wpr;
-      *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, 4 * w, p.katoms)) = 0u;
-      if (w == 0) p.mu[r] = 0.f;
+    // rows M .. m_pad-1 of the last 128-row group: zero scales (finite values for the GEMM)
+    if (!DEBUG_XT) {
+      const int wpr = nb_pad / 4;
+      const int pad_rows = p.m_pad - p.M;
+      const int nthr = NWc * 32;
+      for (int i = blockIdx.x * nthr + tid; i < pad_rows * wpr; i += gridDim.x * nthr) {
+        const int r = p.M + i / wpr, w = i % wpr;
+        *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, 4 * w, p.katoms)) = 0u;
+        if (w == 0) p.mu[r] = 0.f;
+      }
     }
   }
 }
@@ -315,32 +419,79 @@ __global__ void k_encode_f32(const float* __restrict__ V, int M, int K, uint8_t*
 }
 
 // ----------------------------------------------------------------------------------
-// k_lowrank_u: U[m, 0..63] = X L1'_hi + X L1'_lo - (center ? rowsum/K : 0) * c1
+// k_lowrank_u: U[m, 0..63] = X L1'_hi + X L1'_lo - mu[m] c1, stored as fp16
 // ----------------------------------------------------------------------------------
+// Grid (M/128, S), S in {1, 2, 4, 8}: CTA (mt, ks) accumulates the 128-row tile over its
+// share of the K chunks. With S > 1 the S CTAs of a tile form a cluster: each stages its
+// fp32 partial in its own shared memory, and CTA ks then sums rows [ks*128/S, ...) over
+// all S partials (distributed shared memory, fixed order: deterministic).
 namespace lowrank {
 constexpr int kStages = 4;
 constexpr int kTileM = 128;
 constexpr int kChunkK = 64;                      // bf16 elements per stage (128 bytes)
 constexpr uint32_t kABytes = kTileM * 128;       // 16 KB
-constexpr uint32_t kBBytes = kUCols * 128;       // 18 KB
+constexpr uint32_t kBBytes = kUCols * 128;       // 16 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kSmemBytes = 1024 + kStages * kStageBytes + 1024;
-constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmemCols = 128;
 }  // namespace lowrank
+
+__device__ __forceinline__ uint32_t f2_to_half2_sat(float a, float b) {
+  a = fminf(fmaxf(a, -65504.f), 65504.f);
+  b = fminf(fmaxf(b, -65504.f), 65504.f);
+  const __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<const uint32_t*>(&h);
+}
+
+// Cluster reduction of the S fp32 partials ([64][128] column-major in each CTA's smem):
+// CTA ks finalises rows [ks*128/S, (ks+1)*128/S); S threads per row, 64/S columns each,
+// summed over the source CTAs in rank order.
+template <int S>
+__device__ __forceinline__ void lowrank_finish(const LowRankParams& p, const float* part, int m0,
+                                               int ks, int t) {
+  constexpr int kRows = 128 / S, kCols = 64 / S;
+  const int rl = ks * kRows + t % kRows;
+  const int j0 = (t / kRows) * kCols;
+  const int row = m0 + rl;
+  float acc[kCols];
+#pragma unroll
+  for (int c = 0; c < kCols; ++c) acc[c] = 0.f;
+#pragma unroll
+  for (int src = 0; src < S; ++src) {
+#pragma unroll
+    for (int c = 0; c < kCols; ++c) {
+      const uint32_t la = smem_u32(part + (j0 + c) * 128 + rl);
+      acc[c] += ld_shared_cluster_f32(mapa_shared(la, static_cast<uint32_t>(src)));
+    }
+  }
+  if (row < p.M) {
+    const float mu = (p.mu != nullptr) ? p.mu[row] : 0.f;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(p.u + static_cast<size_t>(row) * kRankPad + j0);
+#pragma unroll
+    for (int c = 0; c < kCols; c += 2)
+      dst[c / 2] = f2_to_half2_sat(acc[c] - mu * p.c1[j0 + c], acc[c + 1] - mu * p.c1[j0 + c + 1]);
+  }
+}
 
 __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ LowRankParams p) {
   using namespace lowrank;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+  // no extra alignment offset: every CTA of a cluster must use the same smem offsets
+  uint8_t* smem = smem_raw;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kStages;
   uint64_t* accf = empty + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   uint8_t* stage0 = smem + 1024;
+  float* part = reinterpret_cast<float*>(stage0);   // [64][128] after the main loop (S > 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kTileM;
+  const int mt = blockIdx.x, ks = blockIdx.y, S = gridDim.y;
+  const int m0 = mt * kTileM;
   const int KT = static_cast<int>(cdiv(p.K, kChunkK));
+  const int k_begin = static_cast<int>((static_cast<int64_t>(KT) * ks) / S);
+  const int k_end = static_cast<int>((static_cast<int64_t>(KT) * (ks + 1)) / S);
+  const int nk = k_end - k_begin;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -357,71 +508,83 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int kt = 0; kt < KT; ++kt) {
-        const int s = kt % kStages;
-        if (kt >= kStages &&
-            !mbar_wait(&empty[s], ((kt / kStages) - 1) & 1, p.err, KQ_DEV_ERR_TIMEOUT_EMPTY))
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % kStages;
+        if (i >= kStages &&
+            !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, p.err, KQ_DEV_ERR_TIMEOUT_EMPTY))
           break;
         uint8_t* a = stage0 + s * kStageBytes;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_2d(a, &p.tmap_x, kt * kChunkK, m0, &full[s]);
-        tma_load_2d(a + kABytes, &p.tmap_l1, kt * kChunkK, 0, &full[s]);
+        tma_load_2d(a, &p.tmap_x, (k_begin + i) * kChunkK, m0, &full[s]);
+        tma_load_2d(a + kABytes, &p.tmap_l1, (k_begin + i) * kChunkK, 0, &full[s]);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(kTileM, kUCols);
-      bool ok = true;
-      for (int kt = 0; kt < KT && ok; ++kt) {
-        const int s = kt % kStages;
-        ok = mbar_wait(&full[s], (kt / kStages) & 1, p.err, KQ_DEV_ERR_TIMEOUT_FULL);
-        if (!ok) break;
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % kStages;
+        if (!mbar_wait(&full[s], (i / kStages) & 1, p.err, KQ_DEV_ERR_TIMEOUT_FULL)) break;
         tc_fence_after();
         const uint32_t a = smem_u32(stage0 + s * kStageBytes);
         const uint32_t b = a + kABytes;
 #pragma unroll
         for (int kk = 0; kk < kChunkK / 16; ++kk)
           mma_bf16(tmem, sdesc_sw128_kmajor(a + 32 * kk), sdesc_sw128_kmajor(b + 32 * kk), idesc,
-                   (kt > 0 || kk > 0) ? 1u : 0u);
+                   (i > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&empty[s]);
       }
       tc_commit(accf);
     }
   } else {
-    // epilogue warps 2..5: TMEM lane quadrant = warp % 4
+    // epilogue warps 2..5: TMEM lane quadrant = warp % 4; thread owns tile row rl
     const int q = warp & 3;
-    const int row = m0 + 32 * q + lane;
-    const bool ok = mbar_wait(accf, 0, p.err, KQ_DEV_ERR_TIMEOUT_ACC);
+    const int rl = 32 * q + lane;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, p.err, KQ_DEV_ERR_TIMEOUT_ACC));
     tc_fence_after();
-    if (ok) {
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
-      uint32_t hi0[32], hi1[32], lo0[32], lo1[32], sm[32];
-      tmem_ld_32x32b_x32(tbase + 0, hi0);
-      tmem_ld_32x32b_x32(tbase + 32, hi1);
-      tmem_ld_32x32b_x32(tbase + 64, lo0);
-      tmem_ld_32x32b_x32(tbase + 96, lo1);
-      tmem_ld_32x32b_x32(tbase + 128, sm);
+    const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
+    float u[64];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t hi[32], lo[32];
+      tmem_ld_32x32b_x32(tbase + 32 * h, hi);
+      tmem_ld_32x32b_x32(tbase + 64 + 32 * h, lo);
       tmem_ld_wait();
-      const float mu = p.center ? __uint_as_float(sm[0]) / static_cast<float>(p.K) : 0.f;
-      if (row < p.M) {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) u[32 * h + j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+    }
+    if (!ok || nk == 0) {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) u[j] = 0.f;
+    }
+    if (S == 1) {
+      const int row = m0 + rl;
+      if (ok && row < p.M) {
+        const float mu = (p.mu != nullptr) ? p.mu[row] : 0.f;
         uint32_t packed[32];
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-          const float a0 = __uint_as_float(hi0[j]) + __uint_as_float(lo0[j]) - mu * p.c1[j];
-          const float a1 = __uint_as_float(hi0[j + 1]) + __uint_as_float(lo0[j + 1]) - mu * p.c1[j + 1];
-          const float b0 = __uint_as_float(hi1[j]) + __uint_as_float(lo1[j]) - mu * p.c1[32 + j];
-          const float b1 = __uint_as_float(hi1[j + 1]) + __uint_as_float(lo1[j + 1]) - mu * p.c1[33 + j];
-          const __nv_bfloat162 pa = __floats2bfloat162_rn(a0, a1);
-          const __nv_bfloat162 pb = __floats2bfloat162_rn(b0, b1);
-          packed[j / 2] = *reinterpret_cast<const uint32_t*>(&pa);
-          packed[16 + j / 2] = *reinterpret_cast<const uint32_t*>(&pb);
-        }
+        for (int j = 0; j < 32; ++j)
+          packed[j] = f2_to_half2_sat(u[2 * j] - mu * p.c1[2 * j], u[2 * j + 1] - mu * p.c1[2 * j + 1]);
         uint4* dst = reinterpret_cast<uint4*>(p.u + static_cast<size_t>(row) * kRankPad);
 #pragma unroll
         for (int v = 0; v < 8; ++v)
           dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
       }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 64; ++j) part[j * 128 + rl] = u[j];   // column-major: conflict-free
     }
+  }
+  if (S > 1) {
+    __syncwarp();
+    cluster_sync();                       // every partial is in place
+    if (warp >= 2) {
+      if (S == 2) lowrank_finish<2>(p, part, m0, ks, threadIdx.x - 64);
+      else if (S == 4) lowrank_finish<4>(p, part, m0, ks, threadIdx.x - 64);
+      else lowrank_finish<8>(p, part, m0, ks, threadIdx.x - 64);
+    }
+    __syncwarp();
+    cluster_sync();                       // no CTA leaves while others still read its smem
   }
   tc_fence_before();
   __syncthreads();
@@ -455,9 +618,7 @@ static cudaError_t launch_rows_t(const QuantParams& p, int num_sms, int block, s
 
 cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sms,
                                  cudaStream_t st) {
-  const int items = p.rows_per_group * (p.K / kBlock);
-  int block = static_cast<int>(align_up(static_cast<size_t>(items), 32));
-  if (block > 512) block = 512;
+  const int block = 32 * (p.consumer_warps + 1);
   const size_t smem = p.smem_bytes;
   const int kind = p.kind, c = p.center ? 1 : 0;
 #define KQ_DISPATCH(KD, C)                                                             \
@@ -485,8 +646,20 @@ cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(k_lowrank_u, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(kSmemBytes));
   if (e != cudaSuccess) return e;
-  const int64_t grid = cdiv(p.M, kTileM);
-  k_lowrank_u<<<static_cast<unsigned>(grid), 192, kSmemBytes, st>>>(p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(cdiv(p.M, kTileM)), static_cast<unsigned>(p.split));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = static_cast<unsigned>(p.split);
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, k_lowrank_u, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
