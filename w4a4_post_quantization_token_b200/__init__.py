@@ -41,7 +41,7 @@ class KQError(RuntimeError):
 
 if not os.path.exists(library_path):
     raise ImportError(f"libkq.so not found at {library_path}; build it with "
-                      "`python -m w4a4_post_quantization_token_b200.build`")
+                      "`python w4a4_post_quantization_token_b200/build.py`")
 lib = ctypes.CDLL(library_path)
 
 

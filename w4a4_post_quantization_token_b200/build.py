@@ -1,6 +1,6 @@
 """Build libkq.so in-tree with nvcc for sm_100a (B200).
 
-    python -m w4a4_post_quantization_token_b200.build [--verbose-ptxas]
+    python w4a4_post_quantization_token_b200/build.py [--force] [--verbose-ptxas]
 
 The library is a plain C-ABI shared object (include/kq.h); the Python package
 loads it with ctypes. No PyTorch headers are involved.
