@@ -156,6 +156,33 @@ kq_status kq_linear_host(const kq_layer_desc *desc, const void *weights, const v
                          void *X_dev, int32_t M, void *Y_host, void *Y_dev, int32_t out_dtype,
                          void *act, size_t act_bytes, kq_stream_t stream);
 
+/* kq_linear without a caller-supplied workspace. This call has no counterpart in the
+ * method's description; it exists for callers that cannot allocate device memory on the
+ * path where the layer runs: a C or C++ host with no caching allocator, a serving loop
+ * that must not call cudaMalloc/cudaFree there (they are slow and can synchronise the
+ * whole device), or a process whose device memory is already handed out to another
+ * allocator. It allocates nothing: the activation workspace is a fixed array of
+ * KQ_NOALLOC_WORKSPACE_BYTES bytes inside this library's device image, created when
+ * the library's module is loaded on a device.
+ *   Limit: kq_act_bytes(desc, M) must not exceed KQ_NOALLOC_WORKSPACE_BYTES, else the
+ *     call returns KQ_ERR_WORKSPACE_TOO_SMALL and enqueues nothing (about 22,000
+ *     tokens for K = 1152, 9,500 for K = 3072, 2,500 for K = 12288 with a low-rank
+ *     branch). Use kq_linear with your own workspace for larger M.
+ *   Set-up: the first call made with a given device current looks up the array's
+ *     address on that device (cudaGetSymbolAddress) and caches it; later calls only
+ *     read the cache. Make that first call before any stream capture begins.
+ *   Sharing: every call on a device uses the same array, and it keeps what the last
+ *     call wrote. Each call clears the error word at its head and rewrites everything
+ *     else it reads. Calls whose work can overlap on the GPU (different streams, or
+ *     different host threads, without ordering between them) race on the array and
+ *     give wrong results: order them on one stream, or use kq_linear.
+ *   The device error word is not exposed; a device-side timeout is not reported here
+ *     (use kq_linear with your own workspace and kq_last_device_error for that).
+ * Arguments, output and errors are otherwise those of kq_linear. */
+#define KQ_NOALLOC_WORKSPACE_BYTES ((size_t)16 << 20)
+kq_status kq_linear_noalloc(const kq_layer_desc *desc, const void *weights, const void *X_bf16,
+                            int32_t M, void *Y, int32_t out_dtype, kq_stream_t stream);
+
 /* GEMM half only, on an activation workspace already filled by kq_quantize_act or
  * kq_act_pack. */
 kq_status kq_gemm(const kq_layer_desc *desc, const void *weights, const void *act, int32_t M,

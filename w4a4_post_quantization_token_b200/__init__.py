@@ -14,7 +14,8 @@ import os
 import numpy as np
 
 __all__ = ["KQError", "Layer", "lib", "library_path", "weights_bytes", "act_bytes",
-           "prepare_ws_bytes", "prepare_weights", "quantize_act", "linear", "linear_host",
+           "prepare_ws_bytes", "prepare_weights", "quantize_act", "linear", "linear_noalloc",
+           "linear_host", "NOALLOC_WORKSPACE_BYTES",
            "gemm", "weights_pack", "weights_unpack", "act_pack", "act_unpack",
            "debug_transform", "debug_encode_f32", "last_device_error", "status_string",
            "OUT_F32", "OUT_BF16", "SYMBOLS"]
@@ -30,7 +31,8 @@ library_path = os.path.join(_HERE, "libkq.so")
 SYMBOLS = ["kq_weights_bytes", "kq_act_bytes", "kq_prepare_ws_bytes", "kq_prepare_weights",
            "kq_quantize_act", "kq_linear", "kq_linear_host", "kq_gemm", "kq_weights_pack",
            "kq_weights_unpack", "kq_act_pack", "kq_act_unpack", "kq_debug_transform",
-           "kq_debug_encode_f32", "kq_last_device_error", "kq_status_string", "kq_version"]
+           "kq_debug_encode_f32", "kq_last_device_error", "kq_status_string", "kq_version",
+           "kq_linear_noalloc"]
 
 
 class KQError(RuntimeError):
@@ -67,6 +69,7 @@ _sigs = {
     "kq_quantize_act": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "kq_linear": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P,
                                  ctypes.c_size_t, _P]),
+    "kq_linear_noalloc": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P]),
     "kq_linear_host": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_int32,
                                       _P, ctypes.c_size_t, _P]),
     "kq_gemm": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P]),
@@ -191,6 +194,20 @@ def linear(layer: Layer, weights, X, Y, act, out_dtype: int = OUT_F32, stream=No
     _need(act, torch.uint8, act_bytes(layer, M), "act")
     _check(lib.kq_linear(layer.desc, _ptr(weights), _ptr(X), M, _ptr(Y), int(out_dtype), _ptr(act),
                          act.numel(), _stream(stream)), "kq_linear")
+
+
+def linear_noalloc(layer: Layer, weights, X, Y, out_dtype: int = OUT_F32, stream=None) -> None:
+    """kq_linear on the library's built-in workspace: no workspace argument, nothing
+    allocated. Calls that can overlap on the GPU share that workspace and race."""
+    import torch
+    M = X.shape[0]
+    _need(X, torch.bfloat16, M * layer.K, "X")
+    _need(Y, torch.bfloat16 if out_dtype == OUT_BF16 else torch.float32, M * layer.N, "Y")
+    _check(lib.kq_linear_noalloc(layer.desc, _ptr(weights), _ptr(X), M, _ptr(Y), int(out_dtype),
+                                 _stream(stream)), "kq_linear_noalloc")
+
+
+NOALLOC_WORKSPACE_BYTES = 16 << 20
 
 
 def linear_host(layer: Layer, weights, X_host, X_dev, Y_host, Y_dev, act,

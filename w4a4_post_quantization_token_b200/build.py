@@ -16,7 +16,7 @@ PKG_DIR = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_PATH = os.path.join(PKG_DIR, "libkq.so")
-SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "prepare.cu", "pack.cu"]
+SOURCES = ["api.cu", "quantize.cu", "gemm.cu", "prepare.cu", "pack.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
