@@ -153,6 +153,48 @@ void rpbh_tables(const kq_layer_desc* d, std::vector<float>* sgn) {
   for (int k = 0; k < d->K; ++k) (*sgn)[k] = d->t.sign[k] < 0 ? -rs : rs;
 }
 
+// The RPBH table image the quantize kernel copies into shared memory (layout.cuh).
+void rpbh_qtab(const kq_layer_desc* d, std::vector<uint8_t>* out) {
+  const int K = d->K, nb = K / kBlock;
+  out->assign(qtab_bytes(K), 0);
+  uint16_t* pt = reinterpret_cast<uint16_t*>(out->data());
+  for (int k = 0; k < K; ++k)
+    pt[swz64(static_cast<uint32_t>(k) * 2u) / 2] =
+        static_cast<uint16_t>(swz64(static_cast<uint32_t>(d->t.perm[k]) * 2u));
+  uint32_t* sm = reinterpret_cast<uint32_t*>(out->data() + static_cast<size_t>(K) * 2);
+  for (int b = 0; b < nb; ++b)
+    for (int w = 0; w < 4; ++w) {
+      uint32_t m = 0;
+      for (int j = 0; j < 8; ++j) m |= (d->t.sign[32 * b + 8 * w + j] < 0 ? 8u : 0u) << (4 * j);
+      sm[4 * b + w] = m;
+    }
+}
+
+// Shape of the quantize kernel's work: rows per unit, warps and slots per warp.
+// A unit's u * K/32 blocks should fill the warp's lanes (>= 85% busy); among the shapes
+// whose slots fit in shared memory take the most warps, then two slots per warp (the
+// next unit loads while this one is computed) over one.
+struct QuantShape { int u = 0, warps = 0, stages = 0; };
+QuantShape choose_quant_shape(int K, size_t slot_avail, int max_warps) {
+  const int nb = K / kBlock;
+  const size_t rstride = align_up(static_cast<size_t>(K) * 2, 512);
+  int u_eff = 32;
+  for (int u = 1; u <= 32; ++u) {
+    const int iters = (u * nb + 31) / 32;
+    if (static_cast<double>(u * nb) >= 0.85 * 32.0 * iters) { u_eff = u; break; }
+  }
+  QuantShape q;
+  for (int warps = max_warps; warps >= 1; warps -= (warps > 4 ? 4 : 1))
+    for (int stages = 2; stages >= 1; --stages)
+      for (int u = u_eff; u >= 1; --u)
+        if (static_cast<size_t>(warps) * stages * u * rstride <= slot_avail) {
+          if (q.warps == 0 || (u == u_eff && q.u != u_eff)) { q.u = u; q.warps = warps; q.stages = stages; }
+          if (u == u_eff) return q;
+          break;
+        }
+  return q;
+}
+
 kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const void* X, int M,
                             uint8_t* act, QuantParams* p, const DeviceInfo& di) {
   std::memset(p, 0, sizeof(*p));
@@ -174,48 +216,30 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   p->M = M; p->K = K; p->m_pad = static_cast<int>(AL.m_pad);
   p->kind = d->t.kind; p->center = d->center;
   p->katoms = sf_katoms(K);
-  // groups of R rows; each row staged in a 512-byte aligned slot (its own 64-byte
-  // swizzle pattern), loaded in boxes of up to 256 lines. Centring: each of the 4
-  // consumer warps owns U whole rows; otherwise the consumers stride over the blocks.
+  // each row is staged in a 512-byte aligned slot row (its own 64-byte swizzle pattern),
+  // loaded in boxes of up to 256 lines
   const uint32_t rstride = static_cast<uint32_t>(align_up(static_cast<size_t>(K) * 2, 512));
-  const int nwc = 4;
-  int U = 1, R = 1;
-  if (d->center) {
-    U = static_cast<int>((64 + nb / 2) / nb);
-    if (U < 1) U = 1;
-    if (U > 16) U = 16;
-    R = nwc * U;
-  } else {
-    R = static_cast<int>((4 * 128 + nb / 2) / nb);
-    if (R < 1) R = 1;
-    if (R > 64) R = 64;
-  }
-  while (R > 1 && static_cast<size_t>(R) * rstride > 96 * 1024) {   // keep a slot <= 96 KB
-    if (d->center) { if (U == 1) break; --U; R = nwc * U; } else { --R; }
-  }
+  if (d->t.kind == KQ_T_RPBH && K * 2 > 65535) return KQ_ERR_UNSUPPORTED_SHAPE;
   int box = 1;
   for (int c = 1; c <= 256 && c <= nb; ++c) if (nb % c == 0) box = c;
-  p->rows_per_group = R;
-  p->rows_per_warp = U;
-  p->consumer_warps = nwc;
   p->box_lines = box;
   p->row_stride = rstride;
   if (!make_tmap(&p->tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, 32,
                  static_cast<uint64_t>(M) * nb, 64, 32, static_cast<uint32_t>(box),
                  CU_TENSOR_MAP_SWIZZLE_64B))
     return KQ_ERR_CUDA;
-  p->tables_off = 1024;
-  const size_t tables = d->t.kind == KQ_T_RPBH ? static_cast<size_t>(K) * 2 + static_cast<size_t>(nb) * 16 : 0;
-  p->bufs_off = align_up(p->tables_off + tables, 1024);
-  const size_t buf_bytes = align_up(static_cast<size_t>(R) * rstride, 1024);
-  // prefer a footprint that lets two CTAs share an SM; fall back to the full budget
-  size_t budget = 113 * 1024;
-  if (p->bufs_off + 2 * buf_bytes > budget) budget = 227 * 1024;
-  if (p->bufs_off + buf_bytes > budget) return KQ_ERR_UNSUPPORTED_SHAPE;
-  p->nbufs = static_cast<int>((budget - p->bufs_off) / buf_bytes);
-  if (p->nbufs > 4) p->nbufs = 4;
-  p->smem_bytes = p->bufs_off + static_cast<size_t>(p->nbufs) * buf_bytes;
-  if (d->t.kind == KQ_T_RPBH && K * 2 > 65535) return KQ_ERR_UNSUPPORTED_SHAPE;
+  p->tables_off = kQTablesMin;
+  p->qtab_bytes = d->t.kind == KQ_T_RPBH ? static_cast<uint32_t>(qtab_bytes(K)) : 0u;
+  p->bufs_off = align_up(p->tables_off + p->qtab_bytes, 1024);
+  constexpr size_t kSmemMax = 227 * 1024;
+  if (p->bufs_off + rstride > kSmemMax) return KQ_ERR_UNSUPPORTED_SHAPE;
+  const QuantShape q = choose_quant_shape(K, kSmemMax - p->bufs_off,
+                                          d->t.kind == KQ_T_KRON ? kQMaxWarpsKron : kQMaxWarps);
+  if (q.warps == 0) return KQ_ERR_UNSUPPORTED_SHAPE;
+  p->unit_rows = q.u;
+  p->consumer_warps = q.warps;
+  p->nbufs = q.stages;
+  p->smem_bytes = p->bufs_off + static_cast<size_t>(q.warps) * q.stages * q.u * rstride;
   (void)di;
   if (act) {
     p->codes = act + AL.codes;
@@ -223,8 +247,7 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
     p->mu = reinterpret_cast<float*>(act + AL.mu);
     p->err = reinterpret_cast<uint32_t*>(act + AL.err);
   }
-  p->perm = reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(weights) + WL.perm);
-  p->sgn = reinterpret_cast<const float*>(static_cast<const uint8_t*>(weights) + WL.sgn);
+  p->qtab = static_cast<const uint8_t*>(weights) + WL.qtab;
   return KQ_OK;
 }
 
@@ -374,11 +397,16 @@ kq_status kq_prepare_weights(const kq_layer_desc* desc, const void* W_bf16, void
   a.perm_host = desc->t.kind == KQ_T_RPBH ? desc->t.perm : nullptr;
   a.sgn_host = desc->t.kind == KQ_T_RPBH ? sgn.data() : nullptr;
   a.stream = reinterpret_cast<cudaStream_t>(stream);
-  switch (run_prepare(a)) {
-    case PrepStatus::Ok: return KQ_OK;
-    case PrepStatus::Solver: return KQ_ERR_CUDA;
-    default: return KQ_ERR_CUDA;
+  if (run_prepare(a) != PrepStatus::Ok) return KQ_ERR_CUDA;
+  if (desc->t.kind == KQ_T_RPBH) {
+    std::vector<uint8_t> qtab;
+    rpbh_qtab(desc, &qtab);
+    if (cudaMemcpyAsync(static_cast<uint8_t*>(weights) + wlayout(desc).qtab, qtab.data(), qtab.size(),
+                        cudaMemcpyHostToDevice, a.stream) != cudaSuccess ||
+        cudaStreamSynchronize(a.stream) != cudaSuccess)
+      return KQ_ERR_CUDA;
   }
+  return KQ_OK;
 }
 
 kq_status kq_quantize_act(const kq_layer_desc* desc, const void* weights, const void* X_bf16,
@@ -460,13 +488,17 @@ kq_status kq_weights_pack(const kq_layer_desc* desc, const void* r_codes, const 
     return KQ_ERR_CUDA;
   if (desc->t.kind == KQ_T_RPBH) {
     std::vector<float> sgn;
+    std::vector<uint8_t> qtab;
     rpbh_tables(desc, &sgn);
+    rpbh_qtab(desc, &qtab);
     if (cudaMemcpyAsync(w + WL.perm, desc->t.perm, static_cast<size_t>(desc->K) * 4,
                         cudaMemcpyHostToDevice, st) != cudaSuccess ||
         cudaMemcpyAsync(w + WL.sgn, sgn.data(), static_cast<size_t>(desc->K) * 4,
-                        cudaMemcpyHostToDevice, st) != cudaSuccess)
+                        cudaMemcpyHostToDevice, st) != cudaSuccess ||
+        cudaMemcpyAsync(w + WL.qtab, qtab.data(), qtab.size(), cudaMemcpyHostToDevice, st) !=
+            cudaSuccess)
       return KQ_ERR_CUDA;
-    if (cudaStreamSynchronize(st) != cudaSuccess) return KQ_ERR_CUDA;   // sgn is a local
+    if (cudaStreamSynchronize(st) != cudaSuccess) return KQ_ERR_CUDA;   // host locals
   }
   return KQ_OK;
 }

@@ -12,20 +12,29 @@
 
 namespace kq {
 
+constexpr int kQMaxWarps = 16;        // warps per quantize CTA
+constexpr int kQMaxWarpsKron = 8;     // Kronecker: the factors take ~100 registers
+constexpr int kQMaxStages = 3;        // slots per consumer warp
+constexpr int kQMuOff = 1024;         // smem offset of the per-warp token means
+constexpr int kQTablesMin = kQMuOff + kQMaxWarps * 32 * 8;
+
 struct QuantParams {
   CUtensorMap tmap_x;          // X viewed as [M * K/32 lines, 32 bf16], 64-byte swizzle
   uint64_t Ap[16];             // Kronecker A as pairs (A[i][k], A[i][k]), index 4 i + k
   uint64_t Bp[32];             // Kronecker B as pairs (B[j][2l], B[j][2l+1]), index 4 j + l
   int M, K, m_pad, kind, center;
-  int rows_per_group, rows_per_warp, consumer_warps, box_lines, nbufs;
+  int unit_rows;               // rows per work unit (one consumer warp at a time)
+  int consumer_warps;          // warps per CTA, <= kQMaxWarps (kQMaxWarpsKron)
+  int box_lines;               // 64-byte lines per TMA box (divides K/32, <= 256)
+  int nbufs;                   // slots per consumer warp (<= kQMaxStages)
   uint32_t row_stride;         // bytes between staged rows (512-byte multiple)
+  uint32_t qtab_bytes;         // RPBH table bytes (K * 2 + K/32 * 16)
   size_t tables_off, bufs_off, smem_bytes;   // dynamic shared memory carve-up
   int64_t katoms;
   uint8_t* codes;              // act codes [M, K/2]
   uint8_t* sf;                 // act scales (tensor-core layout)
   float* mu;                   // [m_pad]
-  const int32_t* perm;         // RPBH gather indices [K]
-  const float* sgn;            // RPBH sign / sqrt(32) [K]
+  const uint8_t* qtab;         // RPBH shared-memory table image (weights buffer)
   float* xt;                   // debug: transformed values [M, K] (debug launch only)
   uint32_t* err;
 };

@@ -35,6 +35,20 @@ __host__ __device__ __forceinline__ size_t sf_offset(int64_t row, int64_t kb, in
          static_cast<size_t>((row % 128) / 32) * 4u + static_cast<size_t>(kb % 4);
 }
 
+// Physical byte offset of logical byte `off` in a buffer written by a TMA load with the
+// 64-byte swizzle (16-byte chunk index XOR address bits 7..8); buffer 512-byte aligned.
+__host__ __device__ __forceinline__ uint32_t swz64(uint32_t off) {
+  return off ^ (((off >> 7) & 3u) << 4);
+}
+
+// RPBH table staged by the quantize kernel: uint16 source offsets (64-byte swizzled row
+// byte offsets of perm[k], stored at the swizzled position of element k), then per
+// 32-element block four 32-bit words whose nibble j of word w has bit 3 set when
+// sign[32 b + 8 w + j] < 0 (the code's sign bit).
+__host__ __device__ constexpr size_t qtab_bytes(int64_t K) {
+  return static_cast<size_t>(K) * 2 + static_cast<size_t>(K / 32) * 16;
+}
+
 struct WeightsLayout {
   int64_t K = 0, N = 0, rank = 0, rp = 0, n_pad = 0;
   bool center = false;
@@ -47,6 +61,7 @@ struct WeightsLayout {
   size_t s = 0;        // f32   [N]          1^T W
   size_t perm = 0;     // int32 [K]          RPBH gather indices
   size_t sgn = 0;      // f32   [K]          RPBH sign[k] / sqrt(32)
+  size_t qtab = 0;     // uint8 [K*2 + K/32*16] RPBH table as the quantize kernel stages it
   size_t total = 0;
 
   __host__ __device__ static WeightsLayout make(int64_t K, int64_t N, int64_t rank, bool center,
@@ -66,6 +81,7 @@ struct WeightsLayout {
     L.s = o;      o = align_up(o + static_cast<size_t>(N) * 4, kAlign);
     L.perm = o;   o = align_up(o + (kind == 2 ? static_cast<size_t>(K) * 4 : 0), kAlign);
     L.sgn = o;    o = align_up(o + (kind == 2 ? static_cast<size_t>(K) * 4 : 0), kAlign);
+    L.qtab = o;   o = align_up(o + (kind == 2 ? qtab_bytes(K) : 0), kAlign);
     L.total = o;
     return L;
   }

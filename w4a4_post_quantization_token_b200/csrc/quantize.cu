@@ -29,11 +29,6 @@ namespace kq {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Physical byte offset of logical byte `off` in a buffer written by a TMA load with the
-// 64-byte swizzle (16-byte chunk index XOR address bits 7..8); buffer 512-byte aligned.
-__device__ __forceinline__ uint32_t swz64(uint32_t off) {
-  return off ^ (((off >> 7) & 3u) << 4);
-}
 
 // Load block b (32 bf16) of a swizzled row buffer into fp32 registers.
 __device__ __forceinline__ void load_block_swz(const uint8_t* row, int b, float (&v)[32]) {
@@ -84,8 +79,8 @@ __device__ __forceinline__ double warp_sum_f64(double x) {
 // Kronecker apply on pairs: v2[4i + jp] = (x[8i+2jp], x[8i+2jp+1]);
 // T[i][l] = sum_j x[8i+j] B[j][l] with Bp[4j + lp] = (B[j][2lp], B[j][2lp+1]);
 // Y[k][l] = sum_i A[i][k] T[i][l] with Ap[4i + k] = (A[i][k], A[i][k]).
-__device__ __forceinline__ void kron_apply2(uint64_t (&v2)[16], const uint64_t* __restrict__ Ap,
-                                            const uint64_t* __restrict__ Bp) {
+__device__ __forceinline__ void kron_apply2(uint64_t (&v2)[16], const uint64_t (&Ap)[16],
+                                            const uint64_t (&Bp)[32]) {
   uint64_t t2[16];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -151,12 +146,12 @@ __device__ __forceinline__ void encode_scaled2(const uint64_t (&v2)[16], float f
                       fmul2(v2[4 * w + 3], ff));
 }
 
-constexpr int kQMaxBufs = 4;
 
 // Transform + encode of one 32-element block (row r of the ring slot, block b). Writes the
 // codes (or, in debug mode, the transformed values) and returns the scale byte.
 template <int KIND, bool CENTER, bool DEBUG_XT>
-__device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const uint8_t* rowb,
+__device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const uint64_t (&Ap)[16],
+                                                   const uint64_t (&Bp)[32], const uint8_t* rowb,
                                                    const uint8_t* tables, int row, int b,
                                                    float mu_hi, float mu_lo) {
   const float rs = 0.17677669529663687f;   // fp32(1 / sqrt(32))
@@ -190,7 +185,7 @@ __device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const u
 #pragma unroll
     for (int q = 0; q < 16; ++q) v2[q] = fsub2(fsub2(v2[q], mh), ml);
   }
-  if (KIND == 1) kron_apply2(v2, p.Ap, p.Bp);
+  if (KIND == 1) kron_apply2(v2, Ap, Bp);
   if (KIND == 2) fwht32_2(v2);
   const uint32_t* signs = reinterpret_cast<const uint32_t*>(tables + static_cast<size_t>(p.K) * 2);
   if (DEBUG_XT) {
@@ -260,137 +255,155 @@ __device__ __forceinline__ void store_scales(const QuantParams& p, bool valid, i
   }
 }
 
-// Warp-specialised: warp NWc (the last) issues TMA loads of R-row groups into a ring of
-// S slots (one 512-byte aligned slot per row); warps 0..NWc-1 consume. A slot is handed
-// back through an mbarrier that every consumer warp arrives on. Centring: each consumer
-// warp owns U whole rows of the group, so a token's mean is a warp-local reduction.
-// Without centring the consumers stride over all blocks of the group.
+// Persistent; every warp is its own pipeline. The work is cut into units of u consecutive
+// token rows (u chosen so that u * K/32 blocks fill the lanes of a warp evenly); unit j
+// belongs to CTA j % gridDim.x, and a CTA's units go round-robin to its warps. Each warp
+// owns a ring of S slots in shared memory and issues its own TMA loads into them (one
+// 512-byte aligned, 64-byte swizzled slot row per token): when it has finished a unit it
+// refills that slot with its unit S further on, so the next units are in flight while it
+// computes and no warp ever waits for another. RPBH gather offsets and sign masks arrive
+// once per CTA, as one bulk copy of a table prepared with the weights; the Kronecker
+// factors live in registers. Centring: the warp forms each row's mean (fp32 block sums,
+// fp64 across blocks), then all u * K/32 blocks of the unit are spread over the lanes.
 template <int KIND, bool CENTER, bool DEBUG_XT>
-__global__ void __launch_bounds__(512, 1) k_quantize_rows(const __grid_constant__ QuantParams p) {
+__global__ void __launch_bounds__(KIND == 1 ? 32 * kQMaxWarpsKron : 32 * kQMaxWarps, 1)
+k_quantize_rows(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int NWc = static_cast<int>(blockDim.x >> 5) - 1;          // consumer warps
+  const int NW = p.consumer_warps;
   const int nb = p.K / kBlock;
   const int nb_pad = static_cast<int>(p.katoms) * 4;
-  const int R = p.rows_per_group;
-  const int U = p.rows_per_warp;                                   // centring only
-  const int items = R * nb;
-  const uint32_t rstride = p.row_stride;
-  const uint32_t buf_bytes = static_cast<uint32_t>(align_up(static_cast<size_t>(R) * rstride, 1024));
+  const int u = p.unit_rows;
   const int S = p.nbufs;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem);             // [S]
-  uint64_t* empty = full + kQMaxBufs;                              // [S]
+  const uint32_t rstride = p.row_stride;
+  const uint32_t slot_bytes = static_cast<uint32_t>(u) * rstride;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);             // [NW * S]
+  uint64_t* tabbar = full + kQMaxWarps * kQMaxStages;
+  float2* wmu = reinterpret_cast<float2*>(smem + kQMuOff) + 32 * warp;   // this warp's means
   uint8_t* tables = smem + p.tables_off;
-  uint8_t* bufs = smem + p.bufs_off;
-  const int ngroups = static_cast<int>(cdiv(p.M, R));
+  uint8_t* wbufs = smem + p.bufs_off + static_cast<size_t>(warp) * S * slot_bytes;
+  const int64_t units = cdiv(p.M, u);
+  const int G = static_cast<int>(gridDim.x);
+  const int64_t nl = (units - blockIdx.x + G - 1) / G;             // this CTA's units
+  uint64_t* wfull = full + warp * S;
 
-  if (tid == 0) {
-    for (int b = 0; b < S; ++b) { mbar_init(&full[b], 1); mbar_init(&empty[b], NWc); }
-    fence_mbar_init();
-    prefetch_tmap(&p.tmap_x);
-  }
-  if (KIND == 2) {
-    uint16_t* pt = reinterpret_cast<uint16_t*>(tables);
-    uint32_t* sm = reinterpret_cast<uint32_t*>(tables + static_cast<size_t>(p.K) * 2);
-    for (int k = tid; k < p.K; k += blockDim.x)
-      pt[swz64(static_cast<uint32_t>(k) * 2u) / 2] =
-          static_cast<uint16_t>(swz64(static_cast<uint32_t>(p.perm[k]) * 2u));
-    for (int b = tid; b < nb; b += blockDim.x)
+  uint64_t Ap[16], Bp[32];
+  if (KIND == 1) {
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        uint32_t m = 0;
-        for (int j = 0; j < 8; ++j) m |= (p.sgn[32 * b + 8 * w + j] < 0.f ? 8u : 0u) << (4 * j);
-        sm[4 * b + w] = m;
-      }
+    for (int i = 0; i < 16; ++i) Ap[i] = p.Ap[i];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) Bp[i] = p.Bp[i];
   }
-  __syncthreads();
 
-  if (warp == NWc) {
-    // ----------------------------------------------------------------- producer
-    if (lane == 0) {
-      int k = 0;
-      for (int g = blockIdx.x; g < ngroups; g += gridDim.x, ++k) {
-        const int s = k % S;
-        if (k >= S && !mbar_wait(&empty[s], ((k / S) - 1) & 1, p.err, KQ_DEV_ERR_TIMEOUT_EMPTY)) break;
-        uint8_t* dst = bufs + static_cast<size_t>(s) * buf_bytes;
-        const int rows = min(R, p.M - g * R);
-        mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(rows) * nb * 64u);
-        for (int r = 0; r < rows; ++r)
-          for (int l = 0; l < nb; l += p.box_lines)
-            tma_load_2d(dst + static_cast<size_t>(r) * rstride + static_cast<size_t>(l) * 64u,
-                        &p.tmap_x, 0, (g * R + r) * nb + l, &full[s]);
+  // load unit l (a multiple of NW away from this warp's first) into slot s
+  auto issue = [&](int64_t l, int s) {
+    const int64_t row0 = (l * G + blockIdx.x) * u;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(u), p.M - row0));
+    uint8_t* dst = wbufs + static_cast<size_t>(s) * slot_bytes;
+    mbar_arrive_expect_tx(&wfull[s], static_cast<uint32_t>(rows) * nb * 64u);
+    for (int r = 0; r < rows; ++r)
+      for (int c = 0; c < nb; c += p.box_lines)
+        tma_load_2d(dst + static_cast<size_t>(r) * rstride + static_cast<size_t>(c) * 64u,
+                    &p.tmap_x, 0, static_cast<int32_t>((row0 + r) * nb + c), &wfull[s]);
+  };
+
+  if (lane == 0) {
+    for (int s = 0; s < S; ++s) mbar_init(&wfull[s], 1);
+    if (warp == 0) mbar_init(tabbar, 1);
+    fence_mbar_init();
+    if (warp == 0) {
+      prefetch_tmap(&p.tmap_x);
+      if (KIND == 2) {
+        mbar_arrive_expect_tx(tabbar, p.qtab_bytes);
+        bulk_load(tables, p.qtab, p.qtab_bytes, tabbar);
       }
     }
-  } else {
-    // ----------------------------------------------------------------- consumers
-    int k = 0;
-    for (int g = blockIdx.x; g < ngroups; g += gridDim.x, ++k) {
-      const int s = k % S;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (k / S) & 1, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
-      if (!ok) break;
-      const uint8_t* gbuf = bufs + static_cast<size_t>(s) * buf_bytes;
-      const int row0 = g * R;
-      if (CENTER) {
-        for (int u = 0; u < U; ++u) {
-          const int r = warp * U + u;
-          const int row = row0 + r;
-          if (row >= p.M) break;                                   // warp-uniform
-          const uint8_t* rowb = gbuf + static_cast<size_t>(r) * rstride;
-          double part = 0.0;
-          for (int b = lane; b < nb; b += 32) {
-            uint64_t acc = 0;
+    for (int s = 0; s < S; ++s)
+      if (warp + static_cast<int64_t>(s) * NW < nl) issue(warp + static_cast<int64_t>(s) * NW, s);
+  }
+  __syncthreads();                                                  // tabbar initialised
+
+  bool ok = true;
+  if (KIND == 2) ok = __all_sync(0xffffffffu, mbar_wait(tabbar, 0, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
+  int64_t k = 0;
+  for (int64_t l = warp; ok && l < nl; l += NW, ++k) {
+    const int s = static_cast<int>(k % S);
+    ok = __all_sync(0xffffffffu,
+                    mbar_wait(&wfull[s], static_cast<uint32_t>(k / S) & 1u, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
+    if (!ok) break;
+    const uint8_t* ub = wbufs + static_cast<size_t>(s) * slot_bytes;
+    const int64_t row0 = (l * G + blockIdx.x) * u;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(u), p.M - row0));
+    if (CENTER) {
+      for (int r = 0; r < rows; ++r) {
+        const uint8_t* rowb = ub + static_cast<size_t>(r) * rstride;
+        double part = 0.0;
+        for (int b = lane; b < nb; b += 32) {
+          uint64_t acc = 0;
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-              const uint4 q = *reinterpret_cast<const uint4*>(rowb + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
-              const uint64_t s0 = fadd2(bf16x2_to_f2(q.x), bf16x2_to_f2(q.y));
-              const uint64_t s1 = fadd2(bf16x2_to_f2(q.z), bf16x2_to_f2(q.w));
-              acc = c == 0 ? fadd2(s0, s1) : fadd2(acc, fadd2(s0, s1));
-            }
-            part += static_cast<double>(f2lo(acc) + f2hi(acc));
+          for (int c = 0; c < 4; ++c) {
+            const uint4 q = *reinterpret_cast<const uint4*>(rowb + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
+            const uint64_t s0 = fadd2(bf16x2_to_f2(q.x), bf16x2_to_f2(q.y));
+            const uint64_t s1 = fadd2(bf16x2_to_f2(q.z), bf16x2_to_f2(q.w));
+            acc = c == 0 ? fadd2(s0, s1) : fadd2(acc, fadd2(s0, s1));
           }
-          const double mu64 = warp_sum_f64(part) / static_cast<double>(p.K);
-          const float mu_hi = static_cast<float>(mu64);
-          const float mu_lo = static_cast<float>(mu64 - static_cast<double>(mu_hi));
-          if (lane == 0) p.mu[row] = mu_hi;
-          const int iters = (nb + 31) / 32;
-          for (int t = 0; t < iters; ++t) {
-            const int b = 32 * t + lane;
-            const bool valid = b < nb;
-            uint32_t sb = 0;
-            if (valid) sb = quantize_block<KIND, CENTER, DEBUG_XT>(p, rowb, tables, row, b, mu_hi, mu_lo);
-            if (!DEBUG_XT) store_scales(p, valid, row, b, nb, nb_pad, sb);
-          }
+          part += static_cast<double>(f2lo(acc) + f2hi(acc));
         }
-      } else {
-        for (int r = warp * 32 + lane; r < R; r += NWc * 32)
-          if (row0 + r < p.M) p.mu[row0 + r] = 0.f;
-        const int span = NWc * 32;
-        const int iters = (items + span - 1) / span;
-        for (int t = 0; t < iters; ++t) {
-          const int i = t * span + warp * 32 + lane;
-          const int r = i / nb, b = i - r * nb;
-          const int row = row0 + r;
-          const bool valid = i < items && row < p.M;
-          uint32_t sb = 0;
-          if (valid)
-            sb = quantize_block<KIND, CENTER, DEBUG_XT>(p, gbuf + static_cast<size_t>(r) * rstride, tables,
-                                                         row, b, 0.f, 0.f);
-          if (!DEBUG_XT) store_scales(p, valid, row, b, nb, nb_pad, sb);
+        const double mu64 = warp_sum_f64(part) / static_cast<double>(p.K);
+        const float mu_hi = static_cast<float>(mu64);
+        const float mu_lo = static_cast<float>(mu64 - static_cast<double>(mu_hi));
+        if (lane == 0) {
+          wmu[r] = make_float2(mu_hi, mu_lo);
+          p.mu[row0 + r] = mu_hi;
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
+    } else if (lane < rows) {
+      p.mu[row0 + lane] = 0.f;
     }
-    // rows M .. m_pad-1 of the last 128-row group: zero scales (finite values for the GEMM)
-    if (!DEBUG_XT) {
-      const int wpr = nb_pad / 4;
-      const int pad_rows = p.m_pad - p.M;
-      const int nthr = NWc * 32;
-      for (int i = blockIdx.x * nthr + tid; i < pad_rows * wpr; i += gridDim.x * nthr) {
-        const int r = p.M + i / wpr, w = i % wpr;
-        *reinterpret_cast<uint32_t*>(p.sf + sf_offset(r, 4 * w, p.katoms)) = 0u;
-        if (w == 0) p.mu[r] = 0.f;
+    // all blocks of the unit over the lanes: item i = (row i / nb, block i % nb)
+    const int items = rows * nb;
+    const int iters = (u * nb + 31) / 32;
+    int r = 0, b = lane;
+    while (b >= nb) { b -= nb; ++r; }
+    for (int t = 0; t < iters; ++t) {
+      const bool valid = 32 * t + lane < items;
+      uint32_t sb = 0;
+      if (valid) {
+        float mh = 0.f, ml = 0.f;
+        if (CENTER) { const float2 m = wmu[r]; mh = m.x; ml = m.y; }
+        sb = quantize_block<KIND, CENTER, DEBUG_XT>(p, Ap, Bp, ub + static_cast<size_t>(r) * rstride,
+                                                    tables, static_cast<int>(row0 + r), b, mh, ml);
       }
+      if (!DEBUG_XT) store_scales(p, valid, static_cast<int>(row0 + r), b, nb, nb_pad, sb);
+      b += 32;
+      while (b >= nb) { b -= nb; ++r; }
+    }
+    // every lane is done with the slot: refill it with this warp's unit S further on
+    __syncwarp();
+    if (lane == 0 && l + static_cast<int64_t>(S) * NW < nl) {
+      fence_async_smem();                   // generic reads of the slot before the async write
+      issue(l + static_cast<int64_t>(S) * NW, s);
+    }
+  }
+  // rows M .. m_pad-1 of the last 128-row group: zero scales (finite values for the GEMM)
+  if (!DEBUG_XT) {
+    const int wpr = nb_pad / 4;
+    const int pad_rows = p.m_pad - p.M;
+    const int nthr = NW * 32;
+    for (int i = blockIdx.x * nthr + tid; i < pad_rows * wpr; i += G * nthr) {
+      const int rr = p.M + i / wpr, w = i % wpr;
+      *reinterpret_cast<uint32_t*>(p.sf + sf_offset(rr, 4 * w, p.katoms)) = 0u;
+      if (w == 0) p.mu[rr] = 0.f;
+    }
+  }
+  // no TMA load may still be writing this CTA's shared memory when it exits: a warp
+  // that stopped early (device error) drains its outstanding slots first
+  if (!ok && lane == 0) {
+    for (int64_t kk = k; kk < k + S; ++kk) {
+      const int64_t ll = warp + kk * NW;
+      if (ll >= nl) break;
+      mbar_wait(&wfull[kk % S], static_cast<uint32_t>(kk / S) & 1u, nullptr, 0);
     }
   }
 }
@@ -604,13 +617,9 @@ static cudaError_t launch_rows_t(const QuantParams& p, int num_sms, int block, s
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, block, smem);
-  if (e != cudaSuccess) return e;
-  if (per_sm < 1) per_sm = 1;
-  const int64_t groups = cdiv(p.M, p.rows_per_group);
-  int64_t grid = static_cast<int64_t>(num_sms) * per_sm;
-  if (grid > groups) grid = groups;
+  const int64_t units = cdiv(p.M, p.unit_rows);
+  int64_t grid = num_sms;
+  if (grid > units) grid = units;
   if (grid < 1) grid = 1;
   fn<<<static_cast<unsigned>(grid), block, smem, st>>>(p);
   return cudaGetLastError();
@@ -618,7 +627,7 @@ static cudaError_t launch_rows_t(const QuantParams& p, int num_sms, int block, s
 
 cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sms,
                                  cudaStream_t st) {
-  const int block = 32 * (p.consumer_warps + 1);
+  const int block = 32 * p.consumer_warps;
   const size_t smem = p.smem_bytes;
   const int kind = p.kind, c = p.center ? 1 : 0;
 #define KQ_DISPATCH(KD, C)                                                             \
