@@ -14,10 +14,14 @@
 //   warp 0     TMA producer: codes tiles (128-byte swizzle) and scale runs (plain bulk
 //              copies) into a kStages-deep ring; then the U / L2^T tiles of the tile.
 //   warp 1     TMEM allocator and single-thread MMA issuer. Two TMEM accumulators
-//              (2 x 192 columns) alternate between tiles, so the epilogue of one tile
-//              overlaps the MMAs of the next. Per k-tile: tcgen05.cp of the scales into
-//              TMEM, then block-scaled MMAs (K = 64 each); per tile: 4 fp16 MMAs for the
-//              low-rank branch; tcgen05.commit frees ring slots / hands over accumulators.
+//              (columns 0 and 192) alternate between tiles, so the epilogue of one tile
+//              overlaps the MMAs of the next. Per k-tile: 4 block-scaled MMAs (K = 64
+//              each); per tile: 4 fp16 MMAs for the low-rank branch; tcgen05.commit frees
+//              ring slots / hands over accumulators.
+//   warp 6     scale copier: per k-tile, tcgen05.cp of the stage's block scales into
+//              that stage's own TMEM scale set, then a commit the MMA issuer waits on
+//              (each tcgen05 instruction costs its issuing thread ~50 cycles, so the
+//              copies and the MMAs are issued from two threads).
 //   warps 2-5  epilogue: tcgen05.ld 32 columns at a time, + mu[m] s[n], convert, write a
 //              128-byte-swizzled staging tile in shared memory, TMA-store it (async).
 // A 192-wide tile whose first row sits in the middle of a 128-row scale atom reads its
@@ -41,22 +45,25 @@ constexpr uint32_t kEpiBuf = 4096;                       // 32 rows x 128 bytes
 constexpr int kEpiBufs = 2;                              // per epilogue warp
 constexpr uint32_t kEpiBytes = 4 * kEpiBufs * kEpiBuf;
 constexpr uint32_t kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes + 1024;
-constexpr uint32_t kAccCols = kBN;                       // one accumulator
-constexpr uint32_t kSFACol = 2 * kBN;                    // 384
-constexpr uint32_t kSFBCol = 2 * kBN + 32;               // 416
+constexpr uint32_t kAccStride = kBN;                     // accumulators at columns 0, 192
+constexpr uint32_t kSFCol = 2 * kBN;                     // 384: one scale set per stage
+constexpr uint32_t kSFSetCols = 24;                      // SFA 8 columns, then SFB 16
+static_assert(kSFCol + kStages * kSFSetCols <= 512, "TMEM columns");
 constexpr uint32_t kTmemCols = 512;
+constexpr int kThreads = 224;                            // 7 warps (roles below)
 static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 }  // namespace gemm
 
 template <bool OUT_BF16>
-__global__ void __launch_bounds__(192, 1) k_gemm_mxf4(const __grid_constant__ GemmParams p) {
+__global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_constant__ GemmParams p) {
   using namespace gemm;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kStages;
-  uint64_t* acc_full = empty + kStages;
+  uint64_t* sf_full = empty + kStages;
+  uint64_t* acc_full = sf_full + kStages;
   uint64_t* acc_empty = acc_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   uint8_t* stage0 = smem + 1024;
@@ -71,7 +78,11 @@ __global__ void __launch_bounds__(192, 1) k_gemm_mxf4(const __grid_constant__ Ge
   const int steps = KT + (lowrank ? 1 : 0);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sf_full[s], 1);
+    }
     for (int b = 0; b < 2; ++b) { mbar_init(&acc_full[b], 1); mbar_init(&acc_empty[b], 4); }
     fence_mbar_init();
     prefetch_tmap(&p.tmap_a);
@@ -126,15 +137,24 @@ __global__ void __launch_bounds__(192, 1) k_gemm_mxf4(const __grid_constant__ Ge
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer
+    // A tcgen05 instruction costs the issuing thread ~50 cycles, so this thread issues
+    // only the MMAs and one commit per k-tile (the scale copies come from warp 6) and
+    // does no other arithmetic: descriptors are built once and advanced by constant
+    // offsets (start address >> 4 sits in the low bits).
     if (lane == 0) {
-      const uint32_t t_sfa = tmem + kSFACol;
-      const uint32_t t_sfb = tmem + kSFBCol;
-      int it = 0, local = 0;
+      const uint32_t st_addr = smem_u32(stage0);
+      const uint64_t adesc0 = sdesc_sw128_kmajor(st_addr);
+      const uint64_t bdesc0 = sdesc_sw128_kmajor(st_addr + kABytes);
+      constexpr uint32_t kStageDesc = kStageBytes >> 4;
+      constexpr uint32_t id0 = idesc_mxf4(kBM, kBN, 0, 0), id2 = idesc_mxf4(kBM, kBN, 2, 2);
+      constexpr uint32_t idf16 = idesc_f16(kBM, kBN);              // U and L2^T are fp16
+      int s = 0;
+      uint32_t ph = 0;
+      int local = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x, ++local) {
         const int nt = tile / MT;
-        const int n0 = nt * kBN;
-        const uint32_t shift = (n0 % 128) ? 2u : 0u;
+        const uint32_t shift = ((nt * kBN) % 128) ? 2u : 0u;
         const int buf = local & 1;
         if (local >= 2 &&
             !mbar_wait(&acc_empty[buf], ((local >> 1) - 1) & 1, p.err, KQ_DEV_ERR_TIMEOUT_ACC)) {
@@ -142,48 +162,80 @@ __global__ void __launch_bounds__(192, 1) k_gemm_mxf4(const __grid_constant__ Ge
           break;
         }
         tc_fence_after();
-        const uint32_t d = tmem + static_cast<uint32_t>(buf) * kAccCols;
-        for (int ks = 0; ks < steps; ++ks, ++it) {
-          const int s = it % kStages;
-          if (!mbar_wait(&full[s], (it / kStages) & 1, p.err, KQ_DEV_ERR_TIMEOUT_FULL)) {
+        const uint32_t d = tmem + static_cast<uint32_t>(buf) * kAccStride;
+        for (int ks = 0; ks < steps; ++ks) {
+          if (!mbar_wait(&sf_full[s], ph, p.err, KQ_DEV_ERR_TIMEOUT_FULL)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a = smem_u32(stage0 + s * kStageBytes);
-          const uint32_t b = a + kABytes;
+          const uint64_t so = static_cast<uint64_t>(s) * kStageDesc;
+          const uint64_t ad = adesc0 + so, bd = bdesc0 + so;
           if (ks < KT) {
-            const uint32_t sfa = b + kBBytes;
-            const uint32_t sfb = sfa + kSFABytes;
-#pragma unroll
-            for (int ka = 0; ka < 2; ++ka) {
-              tmem_cp_32x128b_warpx4(t_sfa + 4 * ka, sdesc_plain_rows16(sfa + 512 * ka));
-              tmem_cp_32x128b_warpx4(t_sfb + 8 * ka, sdesc_plain_rows16(sfb + 512 * ka));
-              tmem_cp_32x128b_warpx4(t_sfb + 8 * ka + 4, sdesc_plain_rows16(sfb + 1024 + 512 * ka));
-            }
-            // K-steps of 64 elements that hold data (the last k-tile may be a partial one)
+            const uint32_t fa = tmem + kSFCol + static_cast<uint32_t>(s) * kSFSetCols;
+            const uint32_t fb = fa + 8 + shift;
+            const uint32_t acc0 = ks > 0 ? 1u : 0u;
             const int rem = p.K - ks * kTileK;
-            const int nkk = rem >= kTileK ? 4 : static_cast<int>(cdiv(rem, 64));
-            for (int kk = 0; kk < nkk; ++kk) {
-              const uint32_t ka = kk >> 1, id = 2u * (kk & 1);
-              const uint32_t idesc = idesc_mxf4(kBM, kBN, id, id);
-              mma_mxf4(d, sdesc_sw128_kmajor(a + 32 * kk), sdesc_sw128_kmajor(b + 32 * kk), idesc,
-                       (t_sfa + 4 * ka) | (id << 30), (t_sfb + 8 * ka + shift) | (id << 30),
-                       (ks > 0 || kk > 0) ? 1u : 0u);
+            if (rem >= kTileK) {
+              mma_mxf4(d, ad, bd, id0, fa, fb, acc0);
+              mma_mxf4(d, ad + 2, bd + 2, id2, fa | (2u << 30), fb | (2u << 30), 1u);
+              mma_mxf4(d, ad + 4, bd + 4, id0, fa + 4, fb + 8, 1u);
+              mma_mxf4(d, ad + 6, bd + 6, id2, (fa + 4) | (2u << 30), (fb + 8) | (2u << 30), 1u);
+            } else {
+              // last, partial k-tile: only the K-steps of 64 that hold data
+              const int nkk = static_cast<int>(cdiv(rem, 64));
+              mma_mxf4(d, ad, bd, id0, fa, fb, acc0);
+              if (nkk > 1) mma_mxf4(d, ad + 2, bd + 2, id2, fa | (2u << 30), fb | (2u << 30), 1u);
+              if (nkk > 2) mma_mxf4(d, ad + 4, bd + 4, id0, fa + 4, fb + 8, 1u);
+              if (nkk > 3)
+                mma_mxf4(d, ad + 6, bd + 6, id2, (fa + 4) | (2u << 30), (fb + 8) | (2u << 30), 1u);
             }
           } else {
-            constexpr uint32_t idesc = idesc_f16(kBM, kBN);      // U and L2^T are fp16
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              mma_bf16(d, sdesc_sw128_kmajor(a + 32 * kk), sdesc_sw128_kmajor(b + 32 * kk), idesc,
-                       1u);
+            for (int kk = 0; kk < 4; ++kk) mma_bf16(d, ad + 2 * kk, bd + 2 * kk, idf16, 1u);
           }
           tc_commit(&empty[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
         }
         tc_commit(&acc_full[buf]);
       }
     }
-  } else {
+  } else if (warp == 6) {
+    // ------------------------------------------------------------- scale copier
+    // Per k-tile: the block scales of the stage go from shared memory into that stage's
+    // own TMEM scale set (SFA atoms k0, k1; SFB row atoms a0, a0+1 for k0, then k1),
+    // then a commit tells the MMA issuer they have landed. A stage's set is rewritten
+    // only after the producer refilled the stage, i.e. after the MMAs that read it.
+    if (lane == 0) {
+      const uint64_t sdesc0 = sdesc_plain_rows16(smem_u32(stage0) + kABytes + kBBytes);
+      constexpr uint32_t kStageDesc = kStageBytes >> 4;
+      int s = 0;
+      uint32_t ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
+        for (int ks = 0; ks < steps; ++ks) {
+          if (!mbar_wait(&full[s], ph, p.err, KQ_DEV_ERR_TIMEOUT_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (ks < KT) {
+            const uint32_t fa = tmem + kSFCol + static_cast<uint32_t>(s) * kSFSetCols;
+            const uint32_t fb = fa + 8;
+            const uint64_t sd = sdesc0 + static_cast<uint64_t>(s) * kStageDesc;
+            tmem_cp_32x128b_warpx4(fa, sd);
+            tmem_cp_32x128b_warpx4(fa + 4, sd + 32);
+            tmem_cp_32x128b_warpx4(fb, sd + 64);
+            tmem_cp_32x128b_warpx4(fb + 4, sd + 128);
+            tmem_cp_32x128b_warpx4(fb + 8, sd + 96);
+            tmem_cp_32x128b_warpx4(fb + 12, sd + 160);
+          }
+          tc_commit(&sf_full[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+      }
+    }
+  } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------- epilogue
     const int q = warp & 3;                               // TMEM lane quadrant
     uint8_t* stg = epi0 + static_cast<uint32_t>(q) * kEpiBufs * kEpiBuf;
@@ -199,7 +251,7 @@ __global__ void __launch_bounds__(192, 1) k_gemm_mxf4(const __grid_constant__ Ge
       tc_fence_after();
       const int row = m0 + 32 * q + lane;
       const float mu = (p.mu != nullptr && row < p.M) ? p.mu[row] : 0.f;
-      const uint32_t tbase = tmem + static_cast<uint32_t>(buf) * kAccCols +
+      const uint32_t tbase = tmem + static_cast<uint32_t>(buf) * kAccStride +
                              (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
       for (int c = 0; c < kBN / 32; ++c) {
@@ -291,7 +343,7 @@ static cudaError_t launch_gemm_t(const GemmParams& p, int num_sms, cudaStream_t 
   if (e != cudaSuccess) return e;
   const int64_t tiles = cdiv(p.M, gemm::kBM) * cdiv(p.N, gemm::kBN);
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  fn<<<grid, 192, gemm::kSmemBytes, st>>>(p);
+  fn<<<grid, gemm::kThreads, gemm::kSmemBytes, st>>>(p);
   return cudaGetLastError();
 }
 
