@@ -48,6 +48,27 @@ def _peaks():
         return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
+def measured_traffic(kernel: str, workload_label: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture
+    (profiles/dram_traffic.json), or None when there is none for this workload or the
+    kernel source has changed since it was taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f).get(kernel)
+        if rec is None or rec.get("workload") != workload_label:
+            return None
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != rec["source_sha256_16"]:
+            return None
+        return int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
 # nominal dense ratio FP4 : BF16 on B200 (9 : 2.25 PFLOP/s)
 FP4_OVER_BF16 = 4.0
 
@@ -352,7 +373,7 @@ def main():
         ach = q_bytes / (q_ms * 1e-3) / 1e9
         roof = {"kernel": "k_quantize_rows+k_lowrank_u", "bound": "hbm", "achieved": ach,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
-    roof["traffic"] = None
+    roof["traffic"] = measured_traffic(roof["kernel"], w.label)
     roof["peak_source"] = peaks["source"] + (" (FP4 = 4 x sustained bf16)" if roof["unit"] == "TFLOP/s" else "")
 
     # end-to-end through the host-buffer entry point (pinned memory, copies timed)
