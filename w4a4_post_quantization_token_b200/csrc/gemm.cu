@@ -99,6 +99,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
   if (warp == 0) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
+      grid_dep_wait();                     // codes, scales and U come from the preceding grids
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
@@ -237,6 +238,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
     }
   } else if (warp >= 2 && warp <= 5) {
     // ------------------------------------------------------------- epilogue
+    grid_dep_wait();                       // mu comes from the quantize grid
     const int q = warp & 3;                               // TMEM lane quadrant
     uint8_t* stg = epi0 + static_cast<uint32_t>(q) * kEpiBufs * kEpiBuf;
     const uint32_t r8 = static_cast<uint32_t>(lane & 7);
@@ -343,7 +345,21 @@ static cudaError_t launch_gemm_t(const GemmParams& p, int num_sms, cudaStream_t 
   if (e != cudaSuccess) return e;
   const int64_t tiles = cdiv(p.M, gemm::kBM) * cdiv(p.N, gemm::kBN);
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
-  fn<<<grid, gemm::kThreads, gemm::kSmemBytes, st>>>(p);
+  // programmatic stream serialization: CTAs may start (barrier init, TMEM allocation,
+  // descriptor prefetch) while the quantize grids finish; every read of their outputs
+  // sits behind griddepcontrol.wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(gemm::kThreads);
+  cfg.dynamicSmemBytes = gemm::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, fn, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -322,6 +322,7 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
       if (warp + static_cast<int64_t>(s) * NW < nl) issue(warp + static_cast<int64_t>(s) * NW, s);
   }
   __syncthreads();                                                  // tabbar initialised
+  grid_dep_launch();                       // the low-rank / GEMM kernel may start its prologue
 
   bool ok = true;
   if (KIND == 2) ok = __all_sync(0xffffffffu, mbar_wait(tabbar, 0, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
@@ -518,6 +519,7 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -554,6 +556,9 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
     const int q = warp & 3;
     const int rl = 32 * q + lane;
     const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, p.err, KQ_DEV_ERR_TIMEOUT_ACC));
+    // the token means come from the quantize grid launched just before this one; every CTA
+    // also waits for it before exiting, so the GEMM's wait on this grid covers both
+    grid_dep_wait();
     tc_fence_after();
     const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
     float u[64];
@@ -660,13 +665,15 @@ cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st) {
   cfg.blockDim = dim3(192);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = static_cast<unsigned>(p.split);
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, k_lowrank_u, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

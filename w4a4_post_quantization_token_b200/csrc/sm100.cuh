@@ -140,6 +140,18 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// ------------------------- programmatic dependent launch ---------------------------
+// Let the next kernel in the stream (launched with programmatic stream serialization)
+// start its CTAs and prologue while this grid is still running.
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Block until the preceding grid has completed and its memory is visible (returns at once
+// for a kernel launched without a programmatic dependency).
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 // ------------------------------- clusters ---------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
