@@ -233,9 +233,21 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   p->bufs_off = align_up(p->tables_off + p->qtab_bytes, 1024);
   constexpr size_t kSmemMax = 227 * 1024;
   if (p->bufs_off + rstride > kSmemMax) return KQ_ERR_UNSUPPORTED_SHAPE;
-  const QuantShape q = choose_quant_shape(K, kSmemMax - p->bufs_off,
-                                          d->t.kind == KQ_T_KRON ? kQMaxWarpsKron : kQMaxWarps);
+  const int max_warps = d->t.kind == KQ_T_KRON ? kQMaxWarpsKron : kQMaxWarps;
+  QuantShape q = choose_quant_shape(K, kSmemMax - p->bufs_off, max_warps);
   if (q.warps == 0) return KQ_ERR_UNSUPPORTED_SHAPE;
+  // With a low-rank branch, prefer a footprint that leaves room for one k_lowrank_u CTA on
+  // the same SM: that kernel is launched as a programmatic dependent and reads the token
+  // means only in its epilogue, so its X stream overlaps this kernel. Exactly 8 warps then:
+  // 256 threads x <= 128 registers plus the low-rank CTA's 192 x ~144 fit the 64 K register
+  // file, and fewer warps would cost this kernel more than the overlap gains.
+  if (d->rank > 0) {
+    const size_t share = kSmemPerSM - 2 * kSmemPerBlockReserved - kLowRankSmemBytes;
+    if (p->bufs_off + rstride <= share) {
+      const QuantShape q2 = choose_quant_shape(K, share - p->bufs_off, max_warps < 8 ? max_warps : 8);
+      if (q2.warps == 8) q = q2;
+    }
+  }
   p->unit_rows = q.u;
   p->consumer_warps = q.warps;
   p->nbufs = q.stages;

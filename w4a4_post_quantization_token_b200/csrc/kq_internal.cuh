@@ -17,6 +17,10 @@ constexpr int kQMaxWarpsKron = 8;     // Kronecker: the factors take ~100 regist
 constexpr int kQMaxStages = 3;        // slots per consumer warp
 constexpr int kQMuOff = 1024;         // smem offset of the per-warp token means
 constexpr int kQTablesMin = kQMuOff + kQMaxWarps * 32 * 8;
+// dynamic shared memory of one k_lowrank_u CTA (3 stages of 32 KB + barriers)
+constexpr size_t kLowRankSmemBytes = 1024 + 3 * 32768 + 1024;
+constexpr size_t kSmemPerSM = 233472;          // B200: 228 KB per SM
+constexpr size_t kSmemPerBlockReserved = 1024; // taken by the driver for every resident CTA
 
 struct QuantParams {
   CUtensorMap tmap_x;          // X viewed as [M * K/32 lines, 32 bf16], 64-byte swizzle

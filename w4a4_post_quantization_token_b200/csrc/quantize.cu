@@ -440,7 +440,7 @@ __global__ void k_encode_f32(const float* __restrict__ V, int M, int K, uint8_t*
 // fp32 partial in its own shared memory, and CTA ks then sums rows [ks*128/S, ...) over
 // all S partials (distributed shared memory, fixed order: deterministic).
 namespace lowrank {
-constexpr int kStages = 4;
+constexpr int kStages = 3;
 constexpr int kTileM = 128;
 constexpr int kChunkK = 64;                      // bf16 elements per stage (128 bytes)
 constexpr uint32_t kABytes = kTileM * 128;       // 16 KB
@@ -448,6 +448,7 @@ constexpr uint32_t kBBytes = kUCols * 128;       // 16 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kSmemBytes = 1024 + kStages * kStageBytes + 1024;
 constexpr uint32_t kTmemCols = 128;
+static_assert(kSmemBytes == kLowRankSmemBytes, "shared-memory footprint the quantize shape leaves room for");
 }  // namespace lowrank
 
 __device__ __forceinline__ uint32_t f2_to_half2_sat(float a, float b) {
