@@ -310,12 +310,16 @@ kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* a
                  static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), 128, bn,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return KQ_ERR_CUDA;
+  // low-rank step: only the first 32 of the 64 stored columns when rank <= 32 (the rest
+  // are zero), as 64-byte rows with the 64-byte swizzle
+  const int lrk = d->rank == 0 ? 0 : (d->rank <= 32 ? 32 : kRankPad);
   if (d->rank > 0) {
+    const CUtensorMapSwizzle sw = lrk == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     if (!make_tmap(&gp.tmap_u, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act + AL.u, kRankPad,
-                   static_cast<uint64_t>(M), kRankPad * 2, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B))
+                   static_cast<uint64_t>(M), kRankPad * 2, static_cast<uint32_t>(lrk), 128, sw))
       return KQ_ERR_CUDA;
     if (!make_tmap(&gp.tmap_l2, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w + WL.l2t, kRankPad,
-                   static_cast<uint64_t>(N), kRankPad * 2, 64, bn, CU_TENSOR_MAP_SWIZZLE_128B))
+                   static_cast<uint64_t>(N), kRankPad * 2, static_cast<uint32_t>(lrk), bn, sw))
       return KQ_ERR_CUDA;
   }
   if (!make_tmap(&gp.tmap_y, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
@@ -329,7 +333,7 @@ kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* a
   gp.s = reinterpret_cast<const float*>(w + WL.s);
   gp.y = Y;
   gp.M = M; gp.N = N; gp.K = K;
-  gp.rank_pad = d->rank > 0 ? kRankPad : 0;
+  gp.rank_pad = lrk;
   gp.katoms = sf_katoms(K);
   gp.err = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(act) + AL.err);
   if (launch_gemm(gp, bf16, di.sms, st) != cudaSuccess) return KQ_ERR_CUDA;

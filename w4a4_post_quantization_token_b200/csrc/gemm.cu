@@ -16,7 +16,8 @@
 //   warp 1     TMEM allocator and single-thread MMA issuer. Two TMEM accumulators
 //              (columns 0 and 192) alternate between tiles, so the epilogue of one tile
 //              overlaps the MMAs of the next. Per k-tile: 4 block-scaled MMAs (K = 64
-//              each); per tile: 4 fp16 MMAs for the low-rank branch; tcgen05.commit frees
+//              each); per tile: 2 or 4 fp16 MMAs (rank <= 32 or <= 64) for the low-rank
+//              branch; tcgen05.commit frees
 //              ring slots / hands over accumulators.
 //   warp 6     scale copier: per k-tile, tcgen05.cp of the stage's block scales into
 //              that stage's own TMEM scale set, then a commit the MMA issuer waits on
@@ -129,7 +130,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
             bulk_load(sfb, sfb_base0 + ko, 1024, &full[s]);
             bulk_load(sfb + 1024, sfb_base1 + ko, 1024, &full[s]);
           } else {
-            mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
+            mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(kBM + kBN) * p.rank_pad * 2u);
             tma_load_2d(a, &p.tmap_u, 0, m0, &full[s]);
             tma_load_2d(b, &p.tmap_l2, 0, n0, &full[s]);
           }
@@ -191,6 +192,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
               if (nkk > 3)
                 mma_mxf4(d, ad + 6, bd + 6, id2, (fa + 4) | (2u << 30), (fb + 8) | (2u << 30), 1u);
             }
+          } else if (p.rank_pad == 32) {
+            const uint32_t a_addr = st_addr + static_cast<uint32_t>(s) * kStageBytes;
+            const uint64_t ad64 = sdesc_sw64_kmajor(a_addr), bd64 = sdesc_sw64_kmajor(a_addr + kABytes);
+            mma_bf16(d, ad64, bd64, idf16, 1u);
+            mma_bf16(d, ad64 + 2, bd64 + 2, idf16, 1u);
           } else {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) mma_bf16(d, ad + 2 * kk, bd + 2 * kk, idf16, 1u);

@@ -56,15 +56,16 @@ struct LowRankParams {
 struct GemmParams {
   CUtensorMap tmap_a;          // act codes [M, K/2] uint8, box 128 x 128, 128-byte swizzle
   CUtensorMap tmap_b;          // residual codes [N, K/2] uint8, box 128 x BN
-  CUtensorMap tmap_u;          // U [M, 64] fp16, box 64 x 128
-  CUtensorMap tmap_l2;         // L2^T [N, 64] fp16, box 64 x BN
+  CUtensorMap tmap_u;          // U [M, 64] fp16, box rank_pad x 128
+  CUtensorMap tmap_l2;         // L2^T [N, 64] fp16, box rank_pad x BN
   CUtensorMap tmap_y;          // Y [M, N] f32 or bf16, box (128 bytes) x 32 rows, 128-byte swizzle
   const uint8_t* sfa;          // act scales (tensor-core layout)
   const uint8_t* sfb;          // residual scales (tensor-core layout, one spare row atom)
   const float* mu;             // [M] or null (no centring)
   const float* s;              // [N]
   void* y;                     // [M, N] f32 or bf16
-  int M, N, K, rank_pad;
+  int M, N, K;
+  int rank_pad;                // low-rank K of the GEMM: 0, 32 (64-byte swizzle) or 64 (128-byte)
   int64_t katoms;
   uint32_t* err;
 };

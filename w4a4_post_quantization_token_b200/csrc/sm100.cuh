@@ -259,6 +259,17 @@ __device__ __forceinline__ uint64_t sdesc_sw128_kmajor(uint32_t smem_addr) {
   d |= static_cast<uint64_t>(2u) << 61;
   return d;
 }
+// K-major operand written by a TMA load with the 64-byte swizzle: 64-byte rows, 8-row
+// groups 512 bytes apart (layout type 4).
+__device__ __forceinline__ uint64_t sdesc_sw64_kmajor(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(512u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(4u) << 61;
+  return d;
+}
 // Un-swizzled K-major matrix of 16-byte rows stored contiguously (8-row core
 // matrices 128 bytes apart): the source of a 32x128b tcgen05.cp.
 __device__ __forceinline__ uint64_t sdesc_plain_rows16(uint32_t smem_addr) {
