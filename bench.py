@@ -48,6 +48,54 @@ def _peaks():
         return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
+def quantize_comparator(kq, torch, args, w, inp, sets, R, dev) -> dict:
+    """The quantize kernel alone (rank 0, no centring) on this workload's M x K, once with a
+    Kronecker block transform and once with SmoothQuant's per-channel scaling, over the same
+    rotating activations (KroQuant section 02 reports its kernel up to 14 % faster than
+    SmoothQuant's on MI350). Times are CUDA-event graph replays, microseconds per call."""
+    from synthetic import make_transform, workload as wl
+    Tk = make_transform(wl(w.index, transform="kron"))
+    Lk = kq.Layer(w.K, w.N, 0, False, Tk)
+    Ls = kq.Layer(w.K, w.N, 0, False, {"kind": "none"})
+    wk = torch.zeros(kq.weights_bytes(Lk), dtype=torch.uint8, device=dev)  # not read (Kronecker)
+    X0 = sets[0]["X"].float()
+    Wf = inp["W"].to(dev).float()
+    tiny = torch.finfo(torch.float32).tiny
+    s = (X0.abs().amax(dim=0).clamp_min(tiny) / Wf.abs().amax(dim=1).clamp_min(tiny)).sqrt()
+    inv_s = (1.0 / s.double()).float().contiguous()
+    acts = [torch.empty(kq.act_bytes(Lk, w.M), dtype=torch.uint8, device=dev) for _ in range(R)]
+    calls = {
+        "kroquant": lambda j: kq.quantize_act(Lk, wk, sets[j]["X"], acts[j]),
+        "smoothquant": lambda j: kq.smooth_quantize_act(Ls, inv_s, sets[j]["X"], acts[j]),
+    }
+    out = {}
+    for name, fn in calls.items():
+        for j in range(R):
+            fn(j)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="relaxed"):
+            for j in range(R):
+                fn(j)
+        g.replay()
+        torch.cuda.synchronize()
+        reps = max(10, min(args.steps, 2000) // R)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        out[name] = a.elapsed_time(b) * 1e3 / (reps * R)
+        del g
+    return {"what": "quantize kernel alone, rank 0, no centring: Kronecker (KroQuant) vs "
+                    "per-channel scaling (SmoothQuant, alpha 0.5), same MXFP4 encoder and pipeline",
+            "shape": f"M={w.M} K={w.K}", "kroquant_us": out["kroquant"],
+            "smoothquant_us": out["smoothquant"],
+            "smoothquant_over_kroquant": out["smoothquant"] / out["kroquant"]}
+
+
 def measured_traffic(kernel: str, workload_label: str):
     """DRAM bytes per launch of `kernel` from the committed ncu capture
     (profiles/dram_traffic.json), or None when there is none for this workload or the
@@ -203,6 +251,8 @@ def main():
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-comparator", action="store_true",
+                    help="skip the KroQuant-vs-SmoothQuant quantize-kernel timing")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -413,6 +463,10 @@ def main():
                "sample": f"first {rows} of {w.M} tokens ({dt:.1f} s, fp64 NumPy, weights "
                          f"prepared beforehand)"}
 
+    comparator = None
+    if not args.no_comparator:
+        comparator = quantize_comparator(kq, torch, args, w, inp, sets, R, dev)
+
     launches_per_step = 2 + (1 if w.rank else 0)
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
@@ -434,6 +488,7 @@ def main():
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
         "prepare_ms": prepare_ms,
+        "comparator": comparator,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)

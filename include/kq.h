@@ -141,6 +141,19 @@ kq_status kq_prepare_weights(const kq_layer_desc *desc, const void *W_bf16, void
 kq_status kq_quantize_act(const kq_layer_desc *desc, const void *weights, const void *X_bf16,
                           int32_t M, void *act, size_t act_bytes, kq_stream_t stream);
 
+/* Comparator of KroQuant section 02 (the SmoothQuant channel-wise scaling its
+ * quantization kernel is measured against): the activation is multiplied per channel by
+ * inv_s (fp32, device, [K]; inv_s[k] = 1/s_k with SmoothQuant's s_k = max|X_k|^a /
+ * max|W_k|^(1-a)), each product rounded to fp32, then MXFP4-encoded along K into the
+ * activation workspace (codes and scales in the layout kq_gemm reads; means set to 0).
+ * Same kernel and pipeline as kq_quantize_act, only the transform differs. The layer
+ * descriptor must have no transform, no centring and rank 0 (else KQ_ERR_INVALID_ARG);
+ * the matching weights are kq_prepare_weights of diag(s) W for that descriptor.
+ * inv_s must be 256-byte aligned. Async on `stream`. */
+kq_status kq_smooth_quantize_act(const kq_layer_desc *desc, const float *inv_s,
+                                 const void *X_bf16, int32_t M, void *act, size_t act_bytes,
+                                 kq_stream_t stream);
+
 /* The whole layer: kq_quantize_act followed by the block-scaled FP4 GEMM with the
  * low-rank (U L2) and rank-1 (mu s) branches fused into its accumulator/epilogue
  * (SVDQuant section 3: low-rank work fused into the 4-bit kernel).

@@ -91,6 +91,17 @@ def test_null_and_alignment_errors_before_any_launch():
     assert kq.lib.kq_debug_encode_f32(ok, M, 33, ok, ok, None) == 2
 
 
+def test_smooth_quantize_rejects_layers_with_a_transform():
+    ok = ctypes.c_void_p(0x100000)
+    L = kq.Layer(64, 64, 0, False, _kron())
+    assert kq.lib.kq_smooth_quantize_act(L.desc, ok, ok, 8, ok, 1 << 20, None) == 1
+    Lc = kq.Layer(64, 64, 0, True, {"kind": "none"})
+    assert kq.lib.kq_smooth_quantize_act(Lc.desc, ok, ok, 8, ok, 1 << 20, None) == 1
+    L0 = kq.Layer(64, 64, 0, False, {"kind": "none"})
+    assert kq.lib.kq_smooth_quantize_act(L0.desc, None, ok, 8, ok, 1 << 20, None) == 1
+    assert kq.lib.kq_smooth_quantize_act(L0.desc, ok, ok, 8, ok, 16, None) == 5
+
+
 def test_status_strings():
     for s in range(9):
         assert kq.status_string(s)

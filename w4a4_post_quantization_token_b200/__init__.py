@@ -14,7 +14,8 @@ import os
 import numpy as np
 
 __all__ = ["KQError", "Layer", "lib", "library_path", "weights_bytes", "act_bytes",
-           "prepare_ws_bytes", "prepare_weights", "quantize_act", "linear", "linear_noalloc",
+           "prepare_ws_bytes", "prepare_weights", "quantize_act", "smooth_quantize_act", "linear",
+           "linear_noalloc",
            "linear_host", "NOALLOC_WORKSPACE_BYTES",
            "gemm", "weights_pack", "weights_unpack", "act_pack", "act_unpack",
            "debug_transform", "debug_encode_f32", "last_device_error", "status_string",
@@ -32,7 +33,7 @@ SYMBOLS = ["kq_weights_bytes", "kq_act_bytes", "kq_prepare_ws_bytes", "kq_prepar
            "kq_quantize_act", "kq_linear", "kq_linear_host", "kq_gemm", "kq_weights_pack",
            "kq_weights_unpack", "kq_act_pack", "kq_act_unpack", "kq_debug_transform",
            "kq_debug_encode_f32", "kq_last_device_error", "kq_status_string", "kq_version",
-           "kq_linear_noalloc"]
+           "kq_linear_noalloc", "kq_smooth_quantize_act"]
 
 
 class KQError(RuntimeError):
@@ -69,6 +70,7 @@ _sigs = {
     "kq_quantize_act": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "kq_linear": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P,
                                  ctypes.c_size_t, _P]),
+    "kq_smooth_quantize_act": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "kq_linear_noalloc": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P]),
     "kq_linear_host": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_int32,
                                       _P, ctypes.c_size_t, _P]),
@@ -184,6 +186,17 @@ def quantize_act(layer: Layer, weights, X, act, stream=None) -> None:
     _need(act, torch.uint8, act_bytes(layer, M), "act")
     _check(lib.kq_quantize_act(layer.desc, _ptr(weights), _ptr(X), M, _ptr(act), act.numel(),
                                _stream(stream)), "kq_quantize_act")
+
+
+def smooth_quantize_act(layer: Layer, inv_s, X, act, stream=None) -> None:
+    """SmoothQuant comparator: per-channel multiply by inv_s (fp32 [K]), then MXFP4."""
+    import torch
+    M = X.shape[0]
+    _need(inv_s, torch.float32, layer.K, "inv_s")
+    _need(X, torch.bfloat16, M * layer.K, "X")
+    _need(act, torch.uint8, act_bytes(layer, M), "act")
+    _check(lib.kq_smooth_quantize_act(layer.desc, _ptr(inv_s), _ptr(X), M, _ptr(act), act.numel(),
+                                      _stream(stream)), "kq_smooth_quantize_act")
 
 
 def linear(layer: Layer, weights, X, Y, act, out_dtype: int = OUT_F32, stream=None) -> None:

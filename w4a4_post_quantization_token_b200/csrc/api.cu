@@ -195,8 +195,11 @@ QuantShape choose_quant_shape(int K, size_t slot_avail, int max_warps) {
   return q;
 }
 
+// inv_s non-null selects the SmoothQuant comparator (kind 3): per-channel multiply by
+// inv_s instead of the layer's block transform (the layer must have none).
 kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const void* X, int M,
-                            uint8_t* act, QuantParams* p, const DeviceInfo& di) {
+                            uint8_t* act, QuantParams* p, const DeviceInfo& di,
+                            const float* inv_s = nullptr) {
   std::memset(p, 0, sizeof(*p));
   const WeightsLayout WL = wlayout(d);
   const ActLayout AL = alayout(d, M);
@@ -214,7 +217,8 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
       for (int l = 0; l < 4; ++l) p->Bp[4 * j + l] = pair(d->t.B[8 * j + 2 * l], d->t.B[8 * j + 2 * l + 1]);
   }
   p->M = M; p->K = K; p->m_pad = static_cast<int>(AL.m_pad);
-  p->kind = d->t.kind; p->center = d->center;
+  p->kind = inv_s ? 3 : d->t.kind; p->center = d->center;
+  p->inv_s = inv_s;
   p->katoms = sf_katoms(K);
   // each row is staged in a 512-byte aligned slot row (its own 64-byte swizzle pattern),
   // loaded in boxes of up to 256 lines
@@ -230,7 +234,8 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
     return KQ_ERR_CUDA;
   p->tables_off = kQTablesMin;
   p->qtab_bytes = d->t.kind == KQ_T_RPBH ? static_cast<uint32_t>(qtab_bytes(K)) : 0u;
-  p->bufs_off = align_up(p->tables_off + p->qtab_bytes, 1024);
+  const size_t table_bytes = inv_s ? static_cast<size_t>(K) * 4 : p->qtab_bytes;
+  p->bufs_off = align_up(p->tables_off + table_bytes, 1024);
   constexpr size_t kSmemMax = 227 * 1024;
   if (p->bufs_off + rstride > kSmemMax) return KQ_ERR_UNSUPPORTED_SHAPE;
   const int max_warps = d->t.kind == KQ_T_KRON ? kQMaxWarpsKron : kQMaxWarps;
@@ -259,7 +264,7 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
     p->mu = reinterpret_cast<float*>(act + AL.mu);
     p->err = reinterpret_cast<uint32_t*>(act + AL.err);
   }
-  p->qtab = static_cast<const uint8_t*>(weights) + WL.qtab;
+  p->qtab = weights ? static_cast<const uint8_t*>(weights) + WL.qtab : nullptr;
   return KQ_OK;
 }
 
@@ -438,6 +443,26 @@ kq_status kq_quantize_act(const kq_layer_desc* desc, const void* weights, const 
   // the error word starts at zero for this call
   if (cudaMemsetAsync(act, 0, 4, st) != cudaSuccess) return KQ_ERR_CUDA;
   return run_quantize(desc, weights, X_bf16, M, static_cast<uint8_t*>(act), st, di);
+}
+
+kq_status kq_smooth_quantize_act(const kq_layer_desc* desc, const float* inv_s,
+                                 const void* X_bf16, int32_t M, void* act, size_t act_bytes,
+                                 kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (desc->t.kind != KQ_T_NONE || desc->center || desc->rank != 0) return KQ_ERR_INVALID_ARG;
+  if (M <= 0 || !inv_s || !X_bf16 || !act) return KQ_ERR_INVALID_ARG;
+  if (!aligned(inv_s) || !aligned(X_bf16) || !aligned(act)) return KQ_ERR_ALIGNMENT;
+  if (act_bytes < alayout(desc, M).total) return KQ_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* a = static_cast<uint8_t*>(act);
+  QuantParams qp;
+  if ((s = fill_quant_params(desc, nullptr, X_bf16, M, a, &qp, di, inv_s)) != KQ_OK) return s;
+  if (cudaMemsetAsync(act, 0, 4, st) != cudaSuccess) return KQ_ERR_CUDA;
+  if (launch_quantize_rows(qp, false, di.sms, st) != cudaSuccess) return KQ_ERR_CUDA;
+  return KQ_OK;
 }
 
 kq_status kq_gemm(const kq_layer_desc* desc, const void* weights, const void* act, int32_t M,

@@ -26,7 +26,8 @@ struct QuantParams {
   CUtensorMap tmap_x;          // X viewed as [M * K/32 lines, 32 bf16], 64-byte swizzle
   uint64_t Ap[16];             // Kronecker A as pairs (A[i][k], A[i][k]), index 4 i + k
   uint64_t Bp[32];             // Kronecker B as pairs (B[j][2l], B[j][2l+1]), index 4 j + l
-  int M, K, m_pad, kind, center;
+  int M, K, m_pad, center;
+  int kind;                    // 0 none, 1 Kronecker, 2 RPBH, 3 per-channel scale
   int unit_rows;               // rows per work unit (one consumer warp at a time)
   int consumer_warps;          // warps per CTA, <= kQMaxWarps (kQMaxWarpsKron)
   int box_lines;               // 64-byte lines per TMA box (divides K/32, <= 256)
@@ -39,6 +40,7 @@ struct QuantParams {
   uint8_t* sf;                 // act scales (tensor-core layout)
   float* mu;                   // [m_pad]
   const uint8_t* qtab;         // RPBH shared-memory table image (weights buffer)
+  const float* inv_s;          // kind 3 (SmoothQuant comparator): fp32 [K] inverse channel scales
   float* xt;                   // debug: transformed values [M, K] (debug launch only)
   uint32_t* err;
 };

@@ -9,7 +9,9 @@
 //    x - mu as (x - mu_hi) - mu_lo in fp32. The block transform runs in registers:
 //    Kronecker A^T X_m B with A, B as kernel parameters (KroQuant commentary, section 02),
 //    or gather + 32-point fast Walsh-Hadamard + sign (OrbitQuant commentary, section 03,
-//    RPBH(X) = X P H D). MXFP4 encoding as in encode.cuh (KroQuant section 03).
+//    RPBH(X) = X P H D), or a per-channel multiply by SmoothQuant inverse scales (the
+//    comparator of KroQuant section 02). MXFP4 encoding as in encode.cuh (KroQuant
+//    section 03).
 //  * k_lowrank_u -- U = X L1' - mu c1 (SVDQuant explainer, section 3: the low-rank branch
 //    runs on the high-precision input) as a tcgen05 bf16 GEMM: TMA loads 128x64 tiles of
 //    X and of [L1'_hi; L1'_lo], the MMA accumulates 128 x 128 in TMEM, the epilogue forms
@@ -180,6 +182,17 @@ __device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const u
       v2[4 * c + 3] = bf16x2_to_f2(q.w);
     }
   }
+  if (KIND == 3) {
+    // per-channel inverse scales of this block: 128-byte line b of the table, 16-byte
+    // chunk c stored at chunk c ^ (b % 8) (consecutive lanes read distinct banks)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const float4 f = *reinterpret_cast<const float4*>(
+          tables + static_cast<uint32_t>(b) * 128u + 16u * (static_cast<uint32_t>(c) ^ (static_cast<uint32_t>(b) & 7u)));
+      v2[2 * c] = fmul2(v2[2 * c], f2pack(f.x, f.y));
+      v2[2 * c + 1] = fmul2(v2[2 * c + 1], f2pack(f.z, f.w));
+    }
+  }
   if (CENTER) {
     const uint64_t mh = f2pack(mu_hi, mu_hi), ml = f2pack(mu_lo, mu_lo);
 #pragma unroll
@@ -320,6 +333,14 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
     }
     for (int s = 0; s < S; ++s)
       if (warp + static_cast<int64_t>(s) * NW < nl) issue(warp + static_cast<int64_t>(s) * NW, s);
+  }
+  if (KIND == 3) {
+    // per-channel inverse scales into 128-byte lines (one per block), chunk-swizzled
+    for (int k4 = tid; k4 < p.K / 4; k4 += blockDim.x) {
+      const uint32_t b = static_cast<uint32_t>(k4 / 8), c = static_cast<uint32_t>(k4 % 8);
+      *reinterpret_cast<float4*>(tables + b * 128u + 16u * (c ^ (b & 7u))) =
+          reinterpret_cast<const float4*>(p.inv_s)[k4];
+    }
   }
   __syncthreads();                                                  // tabbar initialised
   grid_dep_launch();                       // the low-rank / GEMM kernel may start its prologue
@@ -641,7 +662,7 @@ cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sm
     return debug_xt ? launch_rows_t<KD, (C != 0), true>(p, num_sms, block, smem, st)   \
                     : launch_rows_t<KD, (C != 0), false>(p, num_sms, block, smem, st);
   KQ_DISPATCH(0, 0) KQ_DISPATCH(0, 1) KQ_DISPATCH(1, 0) KQ_DISPATCH(1, 1) KQ_DISPATCH(2, 0)
-  KQ_DISPATCH(2, 1)
+  KQ_DISPATCH(2, 1) KQ_DISPATCH(3, 0)
 #undef KQ_DISPATCH
   return cudaErrorInvalidValue;
 }
