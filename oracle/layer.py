@@ -31,6 +31,7 @@ Output (``linear``):
 import numpy as np
 
 from . import bf16 as _bf16
+from . import lpfit as _lp
 from . import mxfp4 as _mx
 from . import transforms as _tr
 
@@ -52,8 +53,11 @@ def truncated_svd_factors(Wp, r: int):
     return Uf[:, :r] * rs[None, :], rs[:, None] * Vt[:r, :], S
 
 
-def prepare(W, T: dict, r: int) -> dict:
-    """Offline weight preparation (steps 5-9). W: [K, N] (bf16 values as float64 or torch)."""
+def prepare(W, T: dict, r: int, lp: float | None = None) -> dict:
+    """Offline weight preparation (steps 5-9). W: [K, N] (bf16 values as float64 or torch).
+
+    lp: encode the residual with the robust l_p scale fit (``oracle.lpfit``, CentriQ)
+    instead of the plain OCP rule; None keeps the plain rule."""
     W = _as_f64(W)
     K, N = W.shape
     s = W.sum(axis=0)
@@ -69,7 +73,10 @@ def prepare(W, T: dict, r: int) -> dict:
     R = Wp - L1 @ L2
     R32 = _bf16.round_f32(R)
     # residual blocks run along K for every output column n: encode R^T [N, K]
-    r_codes, r_scales = _mx.encode(R32.T)
+    if lp is None:
+        r_codes, r_scales = _mx.encode(R32.T)
+    else:
+        r_codes, r_scales, _ = _lp.encode_lp(R32.T, lp)
     L1p = _tr.forward_fold(L1, T)
     c1 = L1p.sum(axis=0)
     return {"s": s, "Wp": Wp, "L1": L1, "L2": L2, "S": S, "R": R, "R32": R32,
