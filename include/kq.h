@@ -130,6 +130,16 @@ size_t kq_prepare_ws_bytes(const kq_layer_desc *desc);
 kq_status kq_prepare_weights(const kq_layer_desc *desc, const void *W_bf16, void *weights,
                              void *ws, size_t ws_bytes, kq_stream_t stream);
 
+/* kq_prepare_weights with the residual's MXFP4 block scales fitted under a robust l_p
+ * objective (CentriQ summary and abstract: weights fitted with an l_p objective that tracks
+ * each group's dense mode while discounting heavy tails). Per 32-element block of R the
+ * candidates are the OCP exponent and the three below it; the codes at each are the usual
+ * round-to-nearest-even, saturating ones; the block keeps the candidate with the smallest
+ * sum |r - deq|^p (float64), ties to the larger exponent. Everything else is as in
+ * kq_prepare_weights (same buffers, same sizes). p in (0, 2], else KQ_ERR_INVALID_ARG. */
+kq_status kq_prepare_weights_lp(const kq_layer_desc *desc, double p, const void *W_bf16,
+                                void *weights, void *ws, size_t ws_bytes, kq_stream_t stream);
+
 /* ---------------------------------------------------------------------------------
  * Online activation quantization (every denoising step, every layer; KroQuant
  * section 01 explains why it must run online). CentriQ abstract (centring),
@@ -248,6 +258,11 @@ kq_status kq_debug_transform(const kq_layer_desc *desc, const void *weights,
  * [M, K/2] and scales [M, K/32] (device). */
 kq_status kq_debug_encode_f32(const float *V, int32_t M, int32_t K, void *codes, void *scales,
                               kq_stream_t stream);
+
+/* The robust l_p block-scale fit alone (as kq_prepare_weights_lp applies it to R), on
+ * float32 rows V [M, K] (device), canonical outputs as kq_debug_encode_f32. p in (0, 2]. */
+kq_status kq_debug_encode_lp_f32(const float *V, int32_t M, int32_t K, double p, void *codes,
+                                 void *scales, kq_stream_t stream);
 
 /* Synchronises `stream`, then maps the workspace's device error word to a status
  * (KQ_OK or KQ_ERR_DEVICE_TIMEOUT) and clears it. */

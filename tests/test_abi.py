@@ -102,6 +102,14 @@ def test_smooth_quantize_rejects_layers_with_a_transform():
     assert kq.lib.kq_smooth_quantize_act(L0.desc, ok, ok, 8, ok, 16, None) == 5
 
 
+def test_lp_entry_points_reject_bad_p():
+    ok = ctypes.c_void_p(0x100000)
+    L = kq.Layer(64, 64, 0, False, _kron())
+    for p in (0.0, -1.0, 2.5, float("nan")):
+        assert kq.lib.kq_prepare_weights_lp(L.desc, p, ok, ok, ok, 1 << 30, None) == 1
+        assert kq.lib.kq_debug_encode_lp_f32(ok, 8, 64, p, ok, ok, None) == 1
+
+
 def test_status_strings():
     for s in range(9):
         assert kq.status_string(s)

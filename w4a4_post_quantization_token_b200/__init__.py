@@ -14,7 +14,7 @@ import os
 import numpy as np
 
 __all__ = ["KQError", "Layer", "lib", "library_path", "weights_bytes", "act_bytes",
-           "prepare_ws_bytes", "prepare_weights", "quantize_act", "smooth_quantize_act", "linear",
+           "prepare_ws_bytes", "prepare_weights", "prepare_weights_lp", "debug_encode_lp_f32", "quantize_act", "smooth_quantize_act", "linear",
            "linear_noalloc",
            "linear_host", "NOALLOC_WORKSPACE_BYTES",
            "gemm", "weights_pack", "weights_unpack", "act_pack", "act_unpack",
@@ -33,7 +33,8 @@ SYMBOLS = ["kq_weights_bytes", "kq_act_bytes", "kq_prepare_ws_bytes", "kq_prepar
            "kq_quantize_act", "kq_linear", "kq_linear_host", "kq_gemm", "kq_weights_pack",
            "kq_weights_unpack", "kq_act_pack", "kq_act_unpack", "kq_debug_transform",
            "kq_debug_encode_f32", "kq_last_device_error", "kq_status_string", "kq_version",
-           "kq_linear_noalloc", "kq_smooth_quantize_act"]
+           "kq_linear_noalloc", "kq_smooth_quantize_act", "kq_prepare_weights_lp",
+           "kq_debug_encode_lp_f32"]
 
 
 class KQError(RuntimeError):
@@ -70,6 +71,9 @@ _sigs = {
     "kq_quantize_act": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "kq_linear": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P,
                                  ctypes.c_size_t, _P]),
+    "kq_prepare_weights_lp": (ctypes.c_int, [_D, ctypes.c_double, _P, _P, _P, ctypes.c_size_t, _P]),
+    "kq_debug_encode_lp_f32": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
+                                              _P, _P, _P]),
     "kq_smooth_quantize_act": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_size_t, _P]),
     "kq_linear_noalloc": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_int32, _P]),
     "kq_linear_host": (ctypes.c_int, [_D, _P, _P, _P, ctypes.c_int32, _P, _P, ctypes.c_int32,
@@ -186,6 +190,22 @@ def quantize_act(layer: Layer, weights, X, act, stream=None) -> None:
     _need(act, torch.uint8, act_bytes(layer, M), "act")
     _check(lib.kq_quantize_act(layer.desc, _ptr(weights), _ptr(X), M, _ptr(act), act.numel(),
                                _stream(stream)), "kq_quantize_act")
+
+
+def prepare_weights_lp(layer: Layer, p: float, W, weights, ws, stream=None) -> None:
+    """prepare_weights with the robust l_p fit of the residual's block scales."""
+    import torch
+    _need(W, torch.bfloat16, layer.K * layer.N, "W")
+    _need(weights, torch.uint8, weights_bytes(layer), "weights")
+    _need(ws, torch.uint8, None, "ws")
+    _check(lib.kq_prepare_weights_lp(layer.desc, float(p), _ptr(W), _ptr(weights), _ptr(ws),
+                                     ws.numel(), _stream(stream)), "kq_prepare_weights_lp")
+
+
+def debug_encode_lp_f32(V, p: float, codes, scales, stream=None) -> None:
+    M, K = V.shape
+    _check(lib.kq_debug_encode_lp_f32(_ptr(V), M, K, float(p), _ptr(codes), _ptr(scales),
+                                      _stream(stream)), "kq_debug_encode_lp_f32")
 
 
 def smooth_quantize_act(layer: Layer, inv_s, X, act, stream=None) -> None:

@@ -348,6 +348,57 @@ kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* a
 }  // namespace
 
 // =====================================================================================
+namespace {
+
+kq_status prepare_weights_impl(const kq_layer_desc* desc, const void* W_bf16, void* weights, void* ws,
+                               size_t ws_bytes, kq_stream_t stream, double lp) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (!W_bf16 || !weights || !ws) return KQ_ERR_INVALID_ARG;
+  if (!aligned(W_bf16) || !aligned(weights) || !aligned(ws)) return KQ_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  const size_t lw = prepare_syevd_lwork(desc->K, desc->N, desc->rank);
+  if (lw == 0) return KQ_ERR_CUDA;
+  if (ws_bytes < PrepareWs::make(desc->K, desc->N, desc->rank, lw).total)
+    return KQ_ERR_WORKSPACE_TOO_SMALL;
+
+  double pinv[32 * 32], pfwd[32 * 32];
+  for (int i = 0; i < 32 * 32; ++i) pinv[i] = pfwd[i] = (i / 32 == i % 32) ? 1.0 : 0.0;
+  if (desc->t.kind == KQ_T_KRON) {
+    double A[16], B[64], Ai[16], Bi[64];
+    for (int i = 0; i < 16; ++i) A[i] = desc->t.A[i];
+    for (int i = 0; i < 64; ++i) B[i] = desc->t.B[i];
+    if (!invert(A, 4, Ai) || !invert(B, 8, Bi)) return KQ_ERR_SINGULAR_TRANSFORM;
+    kron32(Ai, Bi, pinv);
+    kron32(A, B, pfwd);
+  }
+  std::vector<float> sgn;
+  if (desc->t.kind == KQ_T_RPBH) rpbh_tables(desc, &sgn);
+
+  PrepareArgs a;
+  a.K = desc->K; a.N = desc->N; a.rank = desc->rank; a.kind = desc->t.kind;
+  a.center = desc->center != 0;
+  a.W = W_bf16; a.weights = weights; a.ws = ws; a.syevd_lwork = lw;
+  a.pinv_host = pinv; a.pfwd_host = pfwd;
+  a.perm_host = desc->t.kind == KQ_T_RPBH ? desc->t.perm : nullptr;
+  a.sgn_host = desc->t.kind == KQ_T_RPBH ? sgn.data() : nullptr;
+  a.stream = reinterpret_cast<cudaStream_t>(stream);
+  a.lp = lp;
+  if (run_prepare(a) != PrepStatus::Ok) return KQ_ERR_CUDA;
+  if (desc->t.kind == KQ_T_RPBH) {
+    std::vector<uint8_t> qtab;
+    rpbh_qtab(desc, &qtab);
+    if (cudaMemcpyAsync(static_cast<uint8_t*>(weights) + wlayout(desc).qtab, qtab.data(), qtab.size(),
+                        cudaMemcpyHostToDevice, a.stream) != cudaSuccess ||
+        cudaStreamSynchronize(a.stream) != cudaSuccess)
+      return KQ_ERR_CUDA;
+  }
+  return KQ_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* kq_status_string(kq_status s) {
@@ -386,48 +437,13 @@ size_t kq_prepare_ws_bytes(const kq_layer_desc* desc) {
 
 kq_status kq_prepare_weights(const kq_layer_desc* desc, const void* W_bf16, void* weights, void* ws,
                              size_t ws_bytes, kq_stream_t stream) {
-  kq_status s = check_desc(desc);
-  if (s != KQ_OK) return s;
-  if (!W_bf16 || !weights || !ws) return KQ_ERR_INVALID_ARG;
-  if (!aligned(W_bf16) || !aligned(weights) || !aligned(ws)) return KQ_ERR_ALIGNMENT;
-  DeviceInfo di;
-  if ((s = current_device(&di)) != KQ_OK) return s;
-  const size_t lw = prepare_syevd_lwork(desc->K, desc->N, desc->rank);
-  if (lw == 0) return KQ_ERR_CUDA;
-  if (ws_bytes < PrepareWs::make(desc->K, desc->N, desc->rank, lw).total)
-    return KQ_ERR_WORKSPACE_TOO_SMALL;
+  return prepare_weights_impl(desc, W_bf16, weights, ws, ws_bytes, stream, 0.0);
+}
 
-  double pinv[32 * 32], pfwd[32 * 32];
-  for (int i = 0; i < 32 * 32; ++i) pinv[i] = pfwd[i] = (i / 32 == i % 32) ? 1.0 : 0.0;
-  if (desc->t.kind == KQ_T_KRON) {
-    double A[16], B[64], Ai[16], Bi[64];
-    for (int i = 0; i < 16; ++i) A[i] = desc->t.A[i];
-    for (int i = 0; i < 64; ++i) B[i] = desc->t.B[i];
-    if (!invert(A, 4, Ai) || !invert(B, 8, Bi)) return KQ_ERR_SINGULAR_TRANSFORM;
-    kron32(Ai, Bi, pinv);
-    kron32(A, B, pfwd);
-  }
-  std::vector<float> sgn;
-  if (desc->t.kind == KQ_T_RPBH) rpbh_tables(desc, &sgn);
-
-  PrepareArgs a;
-  a.K = desc->K; a.N = desc->N; a.rank = desc->rank; a.kind = desc->t.kind;
-  a.center = desc->center != 0;
-  a.W = W_bf16; a.weights = weights; a.ws = ws; a.syevd_lwork = lw;
-  a.pinv_host = pinv; a.pfwd_host = pfwd;
-  a.perm_host = desc->t.kind == KQ_T_RPBH ? desc->t.perm : nullptr;
-  a.sgn_host = desc->t.kind == KQ_T_RPBH ? sgn.data() : nullptr;
-  a.stream = reinterpret_cast<cudaStream_t>(stream);
-  if (run_prepare(a) != PrepStatus::Ok) return KQ_ERR_CUDA;
-  if (desc->t.kind == KQ_T_RPBH) {
-    std::vector<uint8_t> qtab;
-    rpbh_qtab(desc, &qtab);
-    if (cudaMemcpyAsync(static_cast<uint8_t*>(weights) + wlayout(desc).qtab, qtab.data(), qtab.size(),
-                        cudaMemcpyHostToDevice, a.stream) != cudaSuccess ||
-        cudaStreamSynchronize(a.stream) != cudaSuccess)
-      return KQ_ERR_CUDA;
-  }
-  return KQ_OK;
+kq_status kq_prepare_weights_lp(const kq_layer_desc* desc, double p, const void* W_bf16,
+                                void* weights, void* ws, size_t ws_bytes, kq_stream_t stream) {
+  if (!(p > 0.0 && p <= 2.0)) return KQ_ERR_INVALID_ARG;
+  return prepare_weights_impl(desc, W_bf16, weights, ws, ws_bytes, stream, p);
 }
 
 kq_status kq_quantize_act(const kq_layer_desc* desc, const void* weights, const void* X_bf16,
@@ -627,6 +643,21 @@ kq_status kq_debug_encode_f32(const float* V, int32_t M, int32_t K, void* codes,
   if (s != KQ_OK) return s;
   if (launch_encode_f32(V, M, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
+kq_status kq_debug_encode_lp_f32(const float* V, int32_t M, int32_t K, double p, void* codes,
+                                 void* scales, kq_stream_t stream) {
+  if (!V || !codes || !scales || M <= 0 || K <= 0 || !(p > 0.0 && p <= 2.0)) return KQ_ERR_INVALID_ARG;
+  if (K % 32 != 0) return KQ_ERR_UNSUPPORTED_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(V) & 15u) || (reinterpret_cast<uintptr_t>(codes) & 15u))
+    return KQ_ERR_ALIGNMENT;
+  DeviceInfo di;
+  kq_status s = current_device(&di);
+  if (s != KQ_OK) return s;
+  if (launch_encode_f32(V, M, K, static_cast<uint8_t*>(codes), static_cast<uint8_t*>(scales),
+                        reinterpret_cast<cudaStream_t>(stream), p) != cudaSuccess)
     return KQ_ERR_CUDA;
   return KQ_OK;
 }

@@ -54,4 +54,55 @@ __device__ __forceinline__ uint32_t mx_encode32(const float (&v)[32], uint32_t (
   return sb;
 }
 
+// Codes of v[0..31] at a given scale byte (same rounding as mx_encode32).
+__device__ __forceinline__ void mx_codes_at(const float (&v)[32], uint32_t sb, uint32_t (&c)[4]) {
+  const float inv = mx_inv_scale(sb);
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e0 = 8 * w + 2 * j;
+      word |= cvt_e2m1x2(v[e0] * inv, v[e0 + 1] * inv) << (8 * j);
+    }
+    c[w] = word;
+  }
+}
+
+// Robust l_p fit of the block scale (CentriQ: weights fitted under an l_p objective that
+// tracks each group's dense mode and discounts heavy tails). Candidates: the OCP byte sb0
+// and sb0 - 1 .. sb0 - 3 (not below 0); codes as mx_encode32 at each; objective
+// sum_k |v_k - deq_k|^p in float64, summed in element order; the smallest wins, ties keep
+// the larger scale. Returns the scale byte, writes the codes.
+__device__ __forceinline__ uint32_t mx_encode32_lp(const float (&v)[32], double p, uint32_t (&c)[4]) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const uint32_t sb0 = mx_scale_byte(amax);
+  const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  uint32_t best_sb = sb0;
+  double best_f = 0.0;
+  for (int d = 0; d <= 3; ++d) {
+    const uint32_t sb = sb0 >= static_cast<uint32_t>(d) ? sb0 - d : 0u;
+    uint32_t cc[4];
+    mx_codes_at(v, sb, cc);
+    const double sc = ldexp(1.0, static_cast<int>(sb) - 127);
+    double f = 0.0;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) {
+      const uint32_t code = (cc[k / 8] >> (4 * (k % 8))) & 0xFu;
+      const double q = ((code & 8u) ? -mag[code & 7u] : mag[code & 7u]) * sc;
+      const double err = fabs(static_cast<double>(v[k]) - q);
+      f += (p == 1.0) ? err : (p == 2.0) ? err * err : pow(err, p);
+    }
+    if (d == 0 || f < best_f) {
+      best_f = f;
+      best_sb = sb;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) c[w] = cc[w];
+    }
+  }
+  return best_sb;
+}
+
 }  // namespace kq

@@ -75,7 +75,7 @@ struct GemmParams {
 cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sms,
                                  cudaStream_t st);
 cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint8_t* scales,
-                              cudaStream_t st);
+                              cudaStream_t st, double lp = 0.0);
 cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st);
 cudaError_t launch_gemm(const GemmParams& p, bool out_bf16, int num_sms, cudaStream_t st);
 int gemm_tile_n();

@@ -17,6 +17,7 @@ struct PrepareArgs {
   const double* pfwd_host;    // 32x32 P block (row-major), host
   const int32_t* perm_host;   // RPBH [K], host
   const float* sgn_host;      // RPBH sign/sqrt(32) [K], host
+  double lp = 0.0;             // > 0: robust l_p fit of the residual's block scales
   cudaStream_t stream;
 };
 

@@ -127,7 +127,7 @@ __global__ void k_round_factors(const double* __restrict__ E, const double* __re
 // codes [N, K/2] and scales (tensor-core layout). One thread per (n, block).
 __global__ void k_encode_residual(const double* __restrict__ R, int K, int N,
                                   uint8_t* __restrict__ codes, uint8_t* __restrict__ sf,
-                                  int64_t katoms) {
+                                  int64_t katoms, double lp) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   const int b = blockIdx.y;
   if (n >= N) return;
@@ -135,7 +135,8 @@ __global__ void k_encode_residual(const double* __restrict__ R, int K, int N,
 #pragma unroll
   for (int j = 0; j < 32; ++j) v[j] = static_cast<float>(R[static_cast<size_t>(32 * b + j) * N + n]);
   uint32_t c[4];
-  const uint32_t sb = mx_encode32(v, c);
+  // plain OCP rule, or the robust l_p scale fit (CentriQ) when lp > 0
+  const uint32_t sb = lp > 0.0 ? mx_encode32_lp(v, lp, c) : mx_encode32(v, c);
   *reinterpret_cast<uint4*>(codes + static_cast<size_t>(n) * (K / 2) + 16 * b) =
       make_uint4(c[0], c[1], c[2], c[3]);
   sf[sf_offset(n, b, katoms)] = static_cast<uint8_t>(sb);
@@ -327,7 +328,7 @@ PrepStatus run_prepare(const PrepareArgs& a) {
     if (status != PrepStatus::Ok) return status;
   }
   k_encode_residual<<<dim3(static_cast<unsigned>(cdiv(N, 128)), K / 32), 128, 0, st>>>(
-      Wp, K, N, w + WL.rcodes, w + WL.rsf, sf_katoms(K));
+      Wp, K, N, w + WL.rcodes, w + WL.rsf, sf_katoms(K), a.lp);
   CK(cudaGetLastError());
   CK(cudaStreamSynchronize(st));
 #undef CK

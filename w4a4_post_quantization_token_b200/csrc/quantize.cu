@@ -431,10 +431,11 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
 }
 
 // ----------------------------------------------------------------------------------
-// k_encode_f32 (debug): encoder alone on float32 rows, canonical outputs
+// k_encode_f32 (debug): encoder alone on float32 rows, canonical outputs (plain OCP rule,
+// or the robust l_p scale fit when lp > 0)
 // ----------------------------------------------------------------------------------
 __global__ void k_encode_f32(const float* __restrict__ V, int M, int K, uint8_t* __restrict__ codes,
-                             uint8_t* __restrict__ scales) {
+                             uint8_t* __restrict__ scales, double lp) {
   const int nb = K / kBlock;
   const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (t >= static_cast<int64_t>(M) * nb) return;
@@ -448,7 +449,7 @@ __global__ void k_encode_f32(const float* __restrict__ V, int M, int K, uint8_t*
     v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
   }
   uint32_t c[4];
-  const uint32_t sb = mx_encode32(v, c);
+  const uint32_t sb = lp > 0.0 ? mx_encode32_lp(v, lp, c) : mx_encode32(v, c);
   *reinterpret_cast<uint4*>(codes + row * (K / 2) + b * 16) = make_uint4(c[0], c[1], c[2], c[3]);
   scales[row * nb + b] = static_cast<uint8_t>(sb);
 }
@@ -668,12 +669,12 @@ cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sm
 }
 
 cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint8_t* scales,
-                              cudaStream_t st) {
+                              cudaStream_t st, double lp) {
   const int64_t n = static_cast<int64_t>(M) * (K / kBlock);
   const int block = 256;
   const int64_t grid = cdiv(n, block);
   if (n == 0) return cudaSuccess;
-  k_encode_f32<<<static_cast<unsigned>(grid), block, 0, st>>>(V, M, K, codes, scales);
+  k_encode_f32<<<static_cast<unsigned>(grid), block, 0, st>>>(V, M, K, codes, scales, lp);
   return cudaGetLastError();
 }
 
