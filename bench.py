@@ -48,6 +48,25 @@ def _peaks():
         return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
+def max_over_ranks(value: float, dist, device) -> float:
+    """The largest of every rank's value (timings are reported as the slowest rank's).
+    Every rank must call it, in the same order as its other collectives."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_rows(M: int, rank: int, world: int) -> tuple[int, int]:
+    """[begin, end) of the token rows rank `rank` owns when a global batch of M tokens is
+    split over `world` replicas (tokens are independent: no exchange is needed)."""
+    base, extra = divmod(M, world)
+    begin = rank * base + min(rank, extra)
+    return begin, begin + base + (1 if rank < extra else 0)
+
+
 def quantize_comparator(kq, torch, args, w, inp, sets, R, dev) -> dict:
     """The quantize kernel alone (rank 0, no centring) on this workload's M x K, once with a
     Kronecker block transform and once with SmoothQuant's per-channel scaling, over the same
@@ -378,11 +397,8 @@ def main():
     t_end.record(stream)
     torch.cuda.synchronize()
     clk = clocks.stop()
-    elapsed_ms = t_start.elapsed_time(t_end)
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_end), dist if world > 1 else None, dev)
     if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
         dist.barrier()
 
     # per-kernel attribution: the same launches, one phase at a time
@@ -444,11 +460,7 @@ def main():
             kq.linear_host(L, s0["w"], Xh, s0["X"], Yh, s0["Y"], s0["act"], odt)
         e1.record()
         torch.cuda.synchronize()
-        e2e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist if world > 1 else None, dev)
         e2e = {"value": w.M * world * args.e2e_steps / (e2e_ms / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(w.M * w.K * 2),
                "d2h_bytes_per_step": int(w.M * w.N * (2 if out_bf16 else 4)),
