@@ -10,7 +10,7 @@
 // the 4-bit kernels); the third is CentriQ's rank-1 full-precision mean restore (abstract).
 //
 // Persistent kernel, one CTA per SM, static round-robin over 128 x 192 output tiles
-// (M fastest). Warp roles:
+// (grouped order, see tile_coords). Warp roles:
 //   warp 0     TMA producer: codes tiles (128-byte swizzle) and scale runs (plain bulk
 //              copies) into a kStages-deep ring; then the U / L2^T tiles of the tile.
 //   warp 1     TMEM allocator and single-thread MMA issuer. Two TMEM accumulators
@@ -55,6 +55,20 @@ constexpr int kThreads = 224;                            // 7 warps (roles below
 static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 }  // namespace gemm
+
+// Tile order: groups of kGroupM row tiles, and inside a group every column tile for each
+// row tile in turn (row tile fastest). A wave of CTAs then covers a few row tiles across all
+// columns, so the activation codes of those rows are re-read from L2 rather than DRAM even
+// when the output stream is larger than L2; the weight tiles are shared by all groups.
+constexpr int kGroupM = 8;
+__device__ __forceinline__ void tile_coords(int tile, int MT, int NT, int& mt, int& nt) {
+  const int per_group = kGroupM * NT;
+  const int g = tile / per_group;
+  const int r = tile - g * per_group;
+  const int gm = min(kGroupM, MT - g * kGroupM);           // rows in this (maybe last) group
+  mt = g * kGroupM + r % gm;
+  nt = r / gm;
+}
 
 template <bool OUT_BF16>
 __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_constant__ GemmParams p) {
@@ -104,7 +118,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
       int it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x) {
-        const int mt = tile % MT, nt = tile / MT;
+        int mt, nt;
+        tile_coords(tile, MT, NT, mt, nt);
         const int m0 = mt * kBM, n0 = nt * kBN;
         const int a0 = n0 / 128;
         const uint8_t* sfa_base = p.sfa + static_cast<size_t>(mt) * p.katoms * 512u;
@@ -155,7 +170,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
       int local = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < T && ok; tile += gridDim.x, ++local) {
-        const int nt = tile / MT;
+        int mt, nt;
+        tile_coords(tile, MT, NT, mt, nt);
         const uint32_t shift = ((nt * kBN) % 128) ? 2u : 0u;
         const int buf = local & 1;
         if (local >= 2 &&
@@ -251,7 +267,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
     int local = 0;
     uint32_t nstore = 0;
     for (int tile = blockIdx.x; tile < T; tile += gridDim.x, ++local) {
-      const int mt = tile % MT, nt = tile / MT;
+      int mt, nt;
+      tile_coords(tile, MT, NT, mt, nt);
       const int m0 = mt * kBM, n0 = nt * kBN;
       const int buf = local & 1;
       const bool ok = __all_sync(0xffffffffu,
