@@ -456,8 +456,8 @@ kq_status kq_quantize_act(const kq_layer_desc* desc, const void* weights, const 
   DeviceInfo di;
   if ((s = current_device(&di)) != KQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  // the error word starts at zero for this call
-  if (cudaMemsetAsync(act, 0, 4, st) != cudaSuccess) return KQ_ERR_CUDA;
+  // the quantize kernel's first thread clears the device error word (no separate memset
+  // node in front of it)
   return run_quantize(desc, weights, X_bf16, M, static_cast<uint8_t*>(act), st, di);
 }
 
@@ -476,7 +476,6 @@ kq_status kq_smooth_quantize_act(const kq_layer_desc* desc, const float* inv_s,
   uint8_t* a = static_cast<uint8_t*>(act);
   QuantParams qp;
   if ((s = fill_quant_params(desc, nullptr, X_bf16, M, a, &qp, di, inv_s)) != KQ_OK) return s;
-  if (cudaMemsetAsync(act, 0, 4, st) != cudaSuccess) return KQ_ERR_CUDA;
   if (launch_quantize_rows(qp, false, di.sms, st) != cudaSuccess) return KQ_ERR_CUDA;
   return KQ_OK;
 }
