@@ -28,41 +28,6 @@ namespace kq {
 // ----------------------------------------------------------------------------------
 // helpers
 // ----------------------------------------------------------------------------------
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-
-// Load block b (32 bf16) of a swizzled row buffer into fp32 registers.
-__device__ __forceinline__ void load_block_swz(const uint8_t* row, int b, float (&v)[32]) {
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const uint32_t off = static_cast<uint32_t>(b) * 64u + 16u * c;
-    const uint4 q = *reinterpret_cast<const uint4*>(row + swz64(off));
-    v[8 * c + 0] = bf16_lo(q.x); v[8 * c + 1] = bf16_hi(q.x);
-    v[8 * c + 2] = bf16_lo(q.y); v[8 * c + 3] = bf16_hi(q.y);
-    v[8 * c + 4] = bf16_lo(q.z); v[8 * c + 5] = bf16_hi(q.z);
-    v[8 * c + 6] = bf16_lo(q.w); v[8 * c + 7] = bf16_hi(q.w);
-  }
-}
-
-// Gather element e of a swizzled row buffer.
-__device__ __forceinline__ float load_elem_swz(const uint8_t* row, int e) {
-  const uint32_t off = static_cast<uint32_t>(e) * 2u;
-  const uint16_t h = *reinterpret_cast<const uint16_t*>(row + swz64(off));
-  return __uint_as_float(static_cast<uint32_t>(h) << 16);
-}
-
-__device__ __forceinline__ float tree_sum32(const float (&v)[32]) {
-  float s[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) s[i] = v[2 * i] + v[2 * i + 1];
-#pragma unroll
-  for (int w = 8; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) s[i] = s[i] + s[i + w];
-  return s[0];
-}
-
 __device__ __forceinline__ double warp_sum_f64(double x) {
 #pragma unroll
   for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);

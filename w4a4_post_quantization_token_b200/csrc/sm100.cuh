@@ -71,24 +71,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   }
 }
 
-// The same bounded wait for threads that are not on the critical path: between polls
-// the thread sleeps, so a waiting warp does not take issue slots from a warp that
-// shares its scheduler (the MMA issuer).
-__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t* err,
-                                                uint32_t code, uint32_t sleep_ns) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    __nanosleep(sleep_ns);
-    if (mbar_try_wait(a, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      if (err) atomicOr(err, code);
-      return false;
-    }
-  }
-}
-
 // ------------------------------- TMA -------------------------------------------
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -309,16 +291,6 @@ __host__ __device__ constexpr uint32_t idesc_mxf4(uint32_t M, uint32_t N, uint32
        | (1u << 23)           // scale format: E8M0
        | ((M >> 4) << 24)     // M / 16
        | (sfa_id << 29);      // A scale-factor byte id
-}
-
-__device__ __forceinline__ uint32_t elect_one() {
-  uint32_t pred = 0;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "elect.sync _|p, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(pred));
-  return pred;
 }
 
 }  // namespace kq
