@@ -245,8 +245,10 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   // the same SM: that kernel is launched as a programmatic dependent and reads the token
   // means only in its epilogue, so its X stream overlaps this kernel. Exactly 8 warps then:
   // 256 threads x <= 128 registers plus the low-rank CTA's 192 x ~144 fit the 64 K register
-  // file, and fewer warps would cost this kernel more than the overlap gains.
-  if (d->rank > 0) {
+  // file, and fewer warps would cost this kernel more than the overlap gains. Not for the
+  // Kronecker transform: that kernel is FMA-bound and 16 warps beat the overlap (measured:
+  // video layer 314 -> 295 us).
+  if (d->rank > 0 && d->t.kind != KQ_T_KRON) {
     const size_t share = kSmemPerSM - 2 * kSmemPerBlockReserved - kLowRankSmemBytes;
     if (p->bufs_off + rstride <= share) {
       const QuantShape q2 = choose_quant_shape(K, share - p->bufs_off, max_warps < 8 ? max_warps : 8);

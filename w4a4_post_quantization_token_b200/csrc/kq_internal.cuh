@@ -13,7 +13,7 @@
 namespace kq {
 
 constexpr int kQMaxWarps = 16;        // warps per quantize CTA
-constexpr int kQMaxWarpsKron = 8;     // Kronecker: the factors take ~100 registers
+constexpr int kQMaxWarpsKron = 16;    // Kronecker (FMA-bound): as many warps as fit
 constexpr int kQMaxStages = 3;        // slots per consumer warp
 constexpr int kQMuOff = 1024;         // smem offset of the per-warp token means
 constexpr int kQTablesMin = kQMuOff + kQMaxWarps * 32 * 8;
