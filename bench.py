@@ -195,21 +195,30 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = None):
-    """Time the CPU oracle's online path (centre, transform, encode, fp64 contraction with
-    both branches) on the first rows of the batch for about budget_s seconds."""
+def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = None, ln=None):
+    """Time the CPU oracle's online path (LayerNorm front-end when on, centre, transform,
+    encode, fp64 contraction with both branches) on the first rows of the batch for about
+    budget_s seconds."""
     from oracle import layer as olayer
     X = inp["X"]
-    olayer.linear(X[:8], inp["T"], w.center, prep)            # warm caches
+    if ln is not None:
+        from oracle import layernorm as oln
+
+        def linear(Xs, T, c, p):
+            Y = oln.layernorm(Xs.double().numpy(), ln["gamma"], ln["beta"], ln["eps"])
+            return olayer.linear(Y, T, c, p)
+    else:
+        linear = olayer.linear
+    linear(X[:8], inp["T"], w.center, prep)                   # warm caches
     t0 = time.perf_counter()
-    olayer.linear(X[:32], inp["T"], w.center, prep)
+    linear(X[:32], inp["T"], w.center, prep)
     per_row = max((time.perf_counter() - t0) / 32, 1e-6)
     rows = int(min(max_rows or w.M, max(32, budget_s / per_row)))
     t0 = time.perf_counter()
     done = 0
     while done < rows:
         n = min(512, rows - done)
-        olayer.linear(X[done:done + n], inp["T"], w.center, prep)
+        linear(X[done:done + n], inp["T"], w.center, prep)
         done += n
     dt = time.perf_counter() - t0
     return done / dt, done, dt
@@ -272,11 +281,16 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-comparator", action="store_true",
                     help="skip the KroQuant-vs-SmoothQuant quantize-kernel timing")
+    ap.add_argument("--center", action="store_true",
+                    help="force per-token centring on (the workload's own setting otherwise)")
+    ap.add_argument("--layernorm", action="store_true",
+                    help="fuse a LayerNorm front-end (seeded gamma, beta) into the layer; "
+                         "implies --center")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
     from synthetic import workload
-    w = workload(args.workload)
+    w = workload(args.workload, **({"center": True} if args.center or args.layernorm else {}))
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -300,7 +314,11 @@ def main():
     from synthetic import make_inputs
 
     inp = make_inputs(w)
-    L = kq.Layer(w.K, w.N, w.rank, w.center, inp["T"])
+    ln = None
+    if args.layernorm:
+        from synthetic import make_layernorm
+        ln = make_layernorm(w)
+    L = kq.Layer(w.K, w.N, w.rank, w.center, inp["T"], layernorm=ln)
     out_bf16 = args.out == "bf16"
     ydt = torch.bfloat16 if out_bf16 else torch.float32
     odt = kq.OUT_BF16 if out_bf16 else kq.OUT_F32
@@ -470,7 +488,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import layer as olayer
         prep = olayer.prepare(inp["W"], inp["T"], w.rank)
-        v, rows, dt = oracle_tokens_per_s(w, inp, prep, budget_s=12.0)
+        v, rows, dt = oracle_tokens_per_s(w, inp, prep, budget_s=12.0, ln=ln)
         cpu = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"first {rows} of {w.M} tokens ({dt:.1f} s, fp64 NumPy, weights "
                          f"prepared beforehand)"}
@@ -487,7 +505,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": w.label, "global_batch": w.M * world, "tokens_per_gpu": w.M,
                    "K": K, "N": N, "transform": w.transform, "center": w.center, "rank": w.rank,
-                   "out_dtype": args.out, "parallelism": f"replicas x{world} (token-sharded)",
+                   "layernorm": ln is not None, "out_dtype": args.out, "parallelism": f"replicas x{world} (token-sharded)",
                    "l2": f"{R} rotating buffer sets of {set_bytes / 1e6:.0f} MB (> L2)",
                    "graph": graph is not None},
         "phases_ms": {"quantize": q_ms, "gemm": g_ms,

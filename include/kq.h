@@ -90,6 +90,23 @@ typedef struct {
   const int8_t *sign;    /* RPBH: host [K] */
 } kq_transform_desc;
 
+/* Optional LayerNorm front-end, fused into the online half (the KroQuant commentary,
+ * section 01: normalisation layers between the blocks are why the transform runs online).
+ * Per token, over the K channels:  y = (x - m) / sqrt(v + eps) * gamma + beta  with
+ * m the mean and v the biased variance; then the layer runs on y (centring, transform,
+ * MXFP4, low-rank branch, mean restore). Requires center == 1 (the normalised token is
+ * centred); not available to kq_smooth_quantize_act. gamma and beta are read only by
+ * kq_prepare_weights / kq_weights_pack, which copy them into the prepared weights with
+ * the low-rank map diag(gamma) L1' and the sums gamma^T L1', beta^T L1' (KQ_ERR_INVALID_ARG
+ * there if a pointer is null or a value is not finite); later calls need on and eps only.
+ * The activation workspace then also holds each token's m and 1/sqrt(v + eps). */
+typedef struct {
+  int32_t on;            /* 1: front-end on */
+  float eps;             /* > 0 */
+  const float *gamma;    /* host [K], per-channel scale */
+  const float *beta;     /* host [K], per-channel shift */
+} kq_layernorm_desc;
+
 /* One linear layer. The same descriptor (same values) must be passed to
  * kq_prepare_weights and to every later call that uses the prepared weights. */
 typedef struct {
@@ -98,6 +115,7 @@ typedef struct {
   int32_t rank;          /* low-rank branch rank r, 0..64 */
   int32_t center;        /* 1: per-token mean centring with rank-1 restore (CentriQ) */
   kq_transform_desc t;
+  kq_layernorm_desc ln;  /* zero-initialised: no front-end */
 } kq_layer_desc;
 
 /* ---------------------------------------------------------------------------------

@@ -24,7 +24,10 @@ Recipe (all draws from ``numpy.random.default_rng(seed)`` in the order below):
    ``B = I + N(0, 0.1)`` (8x8), drawn from ``default_rng(seed + 1000 * t)`` for
    attempt ``t = 1, 2, ...`` until both condition numbers are below 100, stored
    as float32; or, for the permuted block-Hadamard transform, a permutation of
-   ``[0, K)`` and Rademacher signs from ``default_rng(seed + 1000)``.
+   ``[0, K)`` and Rademacher signs from ``default_rng(seed + 1000)``;
+8. LayerNorm front-end parameters (only where a case asks for them), from
+   ``default_rng(seed + 2000)``: ``gamma = 1 + 0.25 N(0, 1)`` then ``beta = 0.5 N(0, 1)``,
+   each ``[K]`` float32, ``eps = 1e-6`` (adaLN-style modulated scale and shift).
 """
 from __future__ import annotations
 
@@ -33,7 +36,7 @@ import dataclasses
 import numpy as np
 
 __all__ = ["Workload", "WORKLOADS", "workload", "make_activations", "make_weight",
-           "make_transform", "make_inputs"]
+           "make_transform", "make_inputs", "make_layernorm"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -140,6 +143,14 @@ def make_transform(w: Workload) -> dict:
     if w.transform == "none":
         return {"kind": "none"}
     raise ValueError(w.transform)
+
+
+def make_layernorm(w: Workload) -> dict:
+    """``{"gamma": float32[K], "beta": float32[K], "eps": 1e-6}`` (recipe step 8)."""
+    rng = np.random.default_rng(w.seed + 2000)
+    gamma = (1.0 + 0.25 * rng.standard_normal(w.K)).astype(np.float32)
+    beta = (0.5 * rng.standard_normal(w.K)).astype(np.float32)
+    return {"gamma": gamma, "beta": beta, "eps": 1e-6}
 
 
 def make_inputs(w: Workload) -> dict:

@@ -34,7 +34,8 @@ def test_library_is_in_tree_and_versioned():
 def test_struct_layout_matches_c():
     # kq_transform_desc: int32 + ptr + int32 + ptr + int32 + ptr + ptr (with padding) = 56
     assert ctypes.sizeof(kq._TransformDesc) == 56
-    assert ctypes.sizeof(kq._LayerDesc) == 16 + 56
+    # + kq_layernorm_desc: int32 + float + ptr + ptr = 24
+    assert ctypes.sizeof(kq._LayerDesc) == 16 + 56 + 24
 
 
 def _kron():
@@ -114,3 +115,32 @@ def test_status_strings():
     for s in range(9):
         assert kq.status_string(s)
     assert "timed out" in kq.status_string(7)
+
+
+def _ln(K, **kw):
+    d = {"gamma": np.ones(K, np.float32), "beta": np.zeros(K, np.float32), "eps": 1e-6}
+    d.update(kw)
+    return d
+
+
+def test_layernorm_descriptor_validation():
+    K, N = 64, 64
+    plain = kq.Layer(K, N, 8, True, _kron())
+    ln = kq.Layer(K, N, 8, True, _kron(), layernorm=_ln(K))
+    # the front-end adds gamma, beta, the kernel table, diag(gamma) L1' and two sums
+    assert kq.weights_bytes(ln) >= kq.weights_bytes(plain) + 8 * K + 12 * K + 2 * 64 * K * 2
+    # and two per-token floats to the activations
+    assert kq.act_bytes(ln, 300) >= kq.act_bytes(plain, 300) + 2 * 384 * 4
+    # it normalises and then centres: centring must be on; eps must be positive and finite
+    assert kq.weights_bytes(kq.Layer(K, N, 8, False, _kron(), layernorm=_ln(K))) == 0
+    for eps in (0.0, -1e-6, float("nan"), float("inf")):
+        assert kq.weights_bytes(kq.Layer(K, N, 8, True, _kron(), layernorm=_ln(K, eps=eps))) == 0
+    # gamma / beta are read (and checked) only where they are written into the weights
+    ok = ctypes.c_void_p(0x100000)
+    bad = kq.Layer(K, N, 8, True, _kron(), layernorm=_ln(K, gamma=np.full(K, np.nan, np.float32)))
+    assert kq.weights_bytes(bad) > 0
+    assert kq.lib.kq_prepare_weights(bad.desc, ok, ok, ok, 1 << 30, None) == 1
+    assert kq.lib.kq_weights_pack(bad.desc, ok, ok, ok, ok, ok, ok, None) == 1
+    # the SmoothQuant comparator has no front-end
+    L0 = kq.Layer(K, N, 0, True, {"kind": "none"}, layernorm=_ln(K))
+    assert kq.lib.kq_smooth_quantize_act(L0.desc, ok, ok, 8, ok, 1 << 20, None) == 1

@@ -56,9 +56,14 @@ class _TransformDesc(ctypes.Structure):
                 ("sign", ctypes.POINTER(ctypes.c_int8))]
 
 
+class _LayerNormDesc(ctypes.Structure):
+    _fields_ = [("on", ctypes.c_int32), ("eps", ctypes.c_float),
+                ("gamma", ctypes.POINTER(ctypes.c_float)), ("beta", ctypes.POINTER(ctypes.c_float))]
+
+
 class _LayerDesc(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("rank", ctypes.c_int32),
-                ("center", ctypes.c_int32), ("t", _TransformDesc)]
+                ("center", ctypes.c_int32), ("t", _TransformDesc), ("ln", _LayerNormDesc)]
 
 
 _P = ctypes.c_void_p
@@ -109,9 +114,12 @@ class Layer:
 
     ``transform`` is ``{"kind": "kron", "A": 4x4, "B": 8x8}``,
     ``{"kind": "rpbh", "perm": int[K], "sign": +-1[K]}`` or ``{"kind": "none"}``.
+    ``layernorm`` (optional) is ``{"gamma": float[K], "beta": float[K], "eps": float}``: the
+    fused LayerNorm front-end (needs ``center``).
     The host arrays are kept alive by this object."""
 
-    def __init__(self, K: int, N: int, rank: int, center: bool, transform: dict):
+    def __init__(self, K: int, N: int, rank: int, center: bool, transform: dict,
+                 layernorm: dict | None = None):
         self.K, self.N, self.rank, self.center = int(K), int(N), int(rank), bool(center)
         self.transform = transform
         kind = _KIND[transform["kind"]]
@@ -130,7 +138,17 @@ class Layer:
             self._keep += [perm, sign]
             t.perm = perm.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
             t.sign = sign.ctypes.data_as(ctypes.POINTER(ctypes.c_int8))
-        self._desc = _LayerDesc(K=self.K, N=self.N, rank=self.rank, center=int(self.center), t=t)
+        ln = _LayerNormDesc(on=0)
+        self.layernorm = layernorm
+        if layernorm is not None:
+            g = np.ascontiguousarray(layernorm["gamma"], dtype=np.float32)
+            b = np.ascontiguousarray(layernorm["beta"], dtype=np.float32)
+            self._keep += [g, b]
+            ln.on, ln.eps = 1, float(layernorm.get("eps", 1e-6))
+            ln.gamma = g.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+            ln.beta = b.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+        self._desc = _LayerDesc(K=self.K, N=self.N, rank=self.rank, center=int(self.center), t=t,
+                                ln=ln)
 
     @property
     def desc(self):

@@ -99,13 +99,77 @@ kq_status check_desc(const kq_layer_desc* d) {
     }
     default: return KQ_ERR_INVALID_ARG;
   }
+  if (d->ln.on != 0) {
+    // the front-end normalises, then the layer centres the normalised token (CentriQ)
+    if (d->ln.on != 1 || d->center != 1) return KQ_ERR_INVALID_ARG;
+    if (!(d->ln.eps > 0.f) || !std::isfinite(d->ln.eps)) return KQ_ERR_INVALID_ARG;
+  }
+  return KQ_OK;
+}
+
+// gamma and beta are read only where they are written into the weights
+kq_status check_ln_values(const kq_layer_desc* d) {
+  if (d->ln.on == 0) return KQ_OK;
+  if (!d->ln.gamma || !d->ln.beta) return KQ_ERR_INVALID_ARG;
+  for (int k = 0; k < d->K; ++k)
+    if (!std::isfinite(d->ln.gamma[k]) || !std::isfinite(d->ln.beta[k])) return KQ_ERR_INVALID_ARG;
   return KQ_OK;
 }
 
 WeightsLayout wlayout(const kq_layer_desc* d) {
-  return WeightsLayout::make(d->K, d->N, d->rank, d->center != 0, d->t.kind);
+  return WeightsLayout::make(d->K, d->N, d->rank, d->center != 0, d->t.kind, d->ln.on != 0);
 }
-ActLayout alayout(const kq_layer_desc* d, int M) { return ActLayout::make(M, d->K, d->rank); }
+ActLayout alayout(const kq_layer_desc* d, int M) {
+  return ActLayout::make(M, d->K, d->rank, d->ln.on != 0);
+}
+
+// LayerNorm table image (layout: ln_table_bytes). Position j of block b holds channel
+// perm[32 b + j] for RPBH (the transform gathers its input), channel 32 b + j otherwise.
+void ln_table(const kq_layer_desc* d, std::vector<uint8_t>* out) {
+  const int K = d->K, nb = K / kBlock;
+  const bool rpbh = d->t.kind == KQ_T_RPBH;
+  out->assign(ln_table_bytes(K, d->t.kind), 0);
+  uint8_t* o = out->data();
+  auto put = [&](size_t at, float v) { std::memcpy(o + at, &v, 4); };
+  for (int b = 0; b < nb; ++b)
+    for (int j = 0; j < kBlock; ++j) {
+      const uint32_t c = static_cast<uint32_t>(j / 4), e = static_cast<uint32_t>(j % 4);
+      const int src = rpbh ? d->t.perm[kBlock * b + j] : kBlock * b + j;
+      const size_t at = static_cast<size_t>(b) * 256 + ln_chunk_off(static_cast<uint32_t>(b), c) + 4 * e;
+      put(at, d->ln.gamma[src]);
+      put(at + 128, d->ln.beta[src]);
+      if (rpbh)
+        put(static_cast<size_t>(K) * 8 + static_cast<size_t>(b) * 128 +
+                ln_chunk_off(static_cast<uint32_t>(b), c) + 4 * e,
+            d->ln.gamma[kBlock * b + j]);
+    }
+  double sb = 0.0;
+  for (int k = 0; k < K; ++k) sb += static_cast<double>(d->ln.beta[k]);
+  const double mean_b = sb / static_cast<double>(K);
+  std::memcpy(o + out->size() - 16, &mean_b, 8);
+}
+
+// Front-end parts of the prepared weights: gamma, beta, the kernel's table and, with a
+// low-rank branch, diag(gamma) L1' and gamma^T L1', beta^T L1' (from the stored L1').
+kq_status write_ln_weights(const kq_layer_desc* d, uint8_t* w, cudaStream_t st) {
+  if (d->ln.on == 0) return KQ_OK;
+  const WeightsLayout WL = wlayout(d);
+  const size_t kb = static_cast<size_t>(d->K) * 4;
+  std::vector<uint8_t> tab;
+  ln_table(d, &tab);
+  if (cudaMemcpyAsync(w + WL.lng, d->ln.gamma, kb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(w + WL.lnb, d->ln.beta, kb, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(w + WL.lntab, tab.data(), tab.size(), cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  if (d->rank > 0 &&
+      launch_ln_fold(reinterpret_cast<const uint16_t*>(w + WL.l1t),
+                     reinterpret_cast<const float*>(w + WL.lng), reinterpret_cast<const float*>(w + WL.lnb),
+                     d->K, reinterpret_cast<uint16_t*>(w + WL.l1gt), reinterpret_cast<float*>(w + WL.cg),
+                     reinterpret_cast<float*>(w + WL.cb), st) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return KQ_ERR_CUDA;   // host table
+  return KQ_OK;
+}
 
 // Gauss-Jordan inverse with partial pivoting (float64); false if singular.
 bool invert(const double* a, int n, double* inv) {
@@ -232,10 +296,20 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
                  static_cast<uint64_t>(M) * nb, 64, 32, static_cast<uint32_t>(box),
                  CU_TENSOR_MAP_SWIZZLE_64B))
     return KQ_ERR_CUDA;
-  p->tables_off = kQTablesMin;
+  const bool ln = d->ln.on != 0;
+  if (ln && inv_s) return KQ_ERR_INVALID_ARG;
+  p->tables_off = ln ? kQTablesMinLn : kQTablesMin;
   p->qtab_bytes = d->t.kind == KQ_T_RPBH ? static_cast<uint32_t>(qtab_bytes(K)) : 0u;
   const size_t table_bytes = inv_s ? static_cast<size_t>(K) * 4 : p->qtab_bytes;
-  p->bufs_off = align_up(p->tables_off + table_bytes, 1024);
+  size_t tables_end = p->tables_off + table_bytes;
+  if (ln) {
+    p->ln = 1;
+    p->ln_eps = static_cast<double>(d->ln.eps);
+    p->lntab_off = static_cast<uint32_t>(align_up(tables_end, 128));
+    p->lntab_bytes = static_cast<uint32_t>(ln_table_bytes(K, d->t.kind));
+    tables_end = p->lntab_off + p->lntab_bytes;
+  }
+  p->bufs_off = align_up(tables_end, 1024);
   constexpr size_t kSmemMax = 227 * 1024;
   if (p->bufs_off + rstride > kSmemMax) return KQ_ERR_UNSUPPORTED_SHAPE;
   const int max_warps = d->t.kind == KQ_T_KRON ? kQMaxWarpsKron : kQMaxWarps;
@@ -265,8 +339,13 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
     p->sf = act + AL.sf;
     p->mu = reinterpret_cast<float*>(act + AL.mu);
     p->err = reinterpret_cast<uint32_t*>(act + AL.err);
+    if (ln) {
+      p->lnm = reinterpret_cast<float*>(act + AL.lnm);
+      p->lnr = reinterpret_cast<float*>(act + AL.lnr);
+    }
   }
   p->qtab = weights ? static_cast<const uint8_t*>(weights) + WL.qtab : nullptr;
+  if (ln) p->lntab = weights ? static_cast<const uint8_t*>(weights) + WL.lntab : nullptr;
   return KQ_OK;
 }
 
@@ -285,11 +364,20 @@ kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* 
                    static_cast<uint64_t>(M), static_cast<uint64_t>(d->K) * 2, 64, 128,
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return KQ_ERR_CUDA;
-    if (!make_tmap(&lp.tmap_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                   static_cast<const uint8_t*>(weights) + WL.l1t, static_cast<uint64_t>(d->K),
-                   kUCols, static_cast<uint64_t>(d->K) * 2, 64, kUCols, CU_TENSOR_MAP_SWIZZLE_128B))
+    const bool ln = d->ln.on != 0;
+    const uint8_t* w = static_cast<const uint8_t*>(weights);
+    if (!make_tmap(&lp.tmap_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w + (ln ? WL.l1gt : WL.l1t),
+                   static_cast<uint64_t>(d->K), kUCols, static_cast<uint64_t>(d->K) * 2, 64, kUCols,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
       return KQ_ERR_CUDA;
-    lp.c1 = reinterpret_cast<const float*>(static_cast<const uint8_t*>(weights) + WL.c1);
+    lp.c1 = reinterpret_cast<const float*>(w + WL.c1);
+    if (ln) {
+      lp.ln = 1;
+      lp.cg = reinterpret_cast<const float*>(w + WL.cg);
+      lp.cb = reinterpret_cast<const float*>(w + WL.cb);
+      lp.lnm = reinterpret_cast<const float*>(act + AL.lnm);
+      lp.lnr = reinterpret_cast<const float*>(act + AL.lnr);
+    }
     lp.mu = d->center ? reinterpret_cast<const float*>(act + AL.mu) : nullptr;
     lp.u = reinterpret_cast<uint16_t*>(act + AL.u);
     lp.M = M; lp.K = d->K; lp.split = u_split(M, d->K);
@@ -356,6 +444,7 @@ kq_status prepare_weights_impl(const kq_layer_desc* desc, const void* W_bf16, vo
                                size_t ws_bytes, kq_stream_t stream, double lp) {
   kq_status s = check_desc(desc);
   if (s != KQ_OK) return s;
+  if ((s = check_ln_values(desc)) != KQ_OK) return s;
   if (!W_bf16 || !weights || !ws) return KQ_ERR_INVALID_ARG;
   if (!aligned(W_bf16) || !aligned(weights) || !aligned(ws)) return KQ_ERR_ALIGNMENT;
   DeviceInfo di;
@@ -396,7 +485,7 @@ kq_status prepare_weights_impl(const kq_layer_desc* desc, const void* W_bf16, vo
         cudaStreamSynchronize(a.stream) != cudaSuccess)
       return KQ_ERR_CUDA;
   }
-  return KQ_OK;
+  return write_ln_weights(desc, static_cast<uint8_t*>(weights), a.stream);
 }
 
 }  // namespace
@@ -468,7 +557,8 @@ kq_status kq_smooth_quantize_act(const kq_layer_desc* desc, const float* inv_s,
                                  kq_stream_t stream) {
   kq_status s = check_desc(desc);
   if (s != KQ_OK) return s;
-  if (desc->t.kind != KQ_T_NONE || desc->center || desc->rank != 0) return KQ_ERR_INVALID_ARG;
+  if (desc->t.kind != KQ_T_NONE || desc->center || desc->rank != 0 || desc->ln.on)
+    return KQ_ERR_INVALID_ARG;
   if (M <= 0 || !inv_s || !X_bf16 || !act) return KQ_ERR_INVALID_ARG;
   if (!aligned(inv_s) || !aligned(X_bf16) || !aligned(act)) return KQ_ERR_ALIGNMENT;
   if (act_bytes < alayout(desc, M).total) return KQ_ERR_WORKSPACE_TOO_SMALL;
@@ -535,6 +625,7 @@ kq_status kq_weights_pack(const kq_layer_desc* desc, const void* r_codes, const 
   if (s != KQ_OK) return s;
   if (!r_codes || !r_scales || !s_col || !weights) return KQ_ERR_INVALID_ARG;
   if (desc->rank > 0 && (!L1p_f32 || !L2_bf16)) return KQ_ERR_INVALID_ARG;
+  if ((s = check_ln_values(desc)) != KQ_OK) return s;
   if (!aligned(weights)) return KQ_ERR_ALIGNMENT;
   DeviceInfo di;
   if ((s = current_device(&di)) != KQ_OK) return s;
@@ -558,7 +649,7 @@ kq_status kq_weights_pack(const kq_layer_desc* desc, const void* r_codes, const 
       return KQ_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return KQ_ERR_CUDA;   // host locals
   }
-  return KQ_OK;
+  return write_ln_weights(desc, w, st);
 }
 
 kq_status kq_weights_unpack(const kq_layer_desc* desc, const void* weights, void* r_codes,

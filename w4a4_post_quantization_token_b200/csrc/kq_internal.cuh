@@ -17,6 +17,9 @@ constexpr int kQMaxWarpsKron = 16;    // Kronecker (FMA-bound): as many warps as
 constexpr int kQMaxStages = 3;        // slots per consumer warp
 constexpr int kQMuOff = 1024;         // smem offset of the per-warp token means
 constexpr int kQTablesMin = kQMuOff + kQMaxWarps * 32 * 8;
+// LayerNorm front-end: per-row float4 (rstd, mean_y hi, mean_y lo, 0) after the means
+constexpr int kQLnOff = kQTablesMin;
+constexpr int kQTablesMinLn = kQLnOff + kQMaxWarps * 32 * 16;
 // dynamic shared memory of one k_lowrank_u CTA (3 stages of 32 KB + barriers)
 constexpr size_t kLowRankSmemBytes = 1024 + 3 * 32768 + 1024;
 constexpr size_t kSmemPerSM = 233472;          // B200: 228 KB per SM
@@ -41,6 +44,13 @@ struct QuantParams {
   float* mu;                   // [m_pad]
   const uint8_t* qtab;         // RPBH shared-memory table image (weights buffer)
   const float* inv_s;          // kind 3 (SmoothQuant comparator): fp32 [K] inverse channel scales
+  int ln;                      // LayerNorm front-end on (needs center)
+  double ln_eps;
+  const uint8_t* lntab;        // LayerNorm table image (weights buffer), ln_table_bytes
+  uint32_t lntab_bytes;
+  uint32_t lntab_off;          // its shared-memory offset (128-byte aligned)
+  float* lnm;                  // out: per-token mean of x [m_pad]
+  float* lnr;                  // out: per-token 1/sqrt(v + eps) [m_pad]
   float* xt;                   // debug: transformed values [M, K] (debug launch only)
   uint32_t* err;
 };
@@ -51,6 +61,11 @@ struct LowRankParams {
   const float* c1;             // [64]
   const float* mu;             // [M] token means (null without centring)
   uint16_t* u;                 // U [M, 64] fp16
+  int ln;                      // LayerNorm front-end: L1 map is diag(gamma) L1', and
+  const float* cg;             //   U = rstd acc - rstd m cg + cb - mu c1 with cg = gamma^T L1'
+  const float* cb;             //   and cb = beta^T L1' [64]
+  const float* lnm;            //   per-token m and rstd from the quantize kernel
+  const float* lnr;
   int M, K, split;             // split: CTAs (one cluster) per 128-row tile, 1/2/4/8
   uint32_t* err;
 };
@@ -77,6 +92,10 @@ cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sm
 cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint8_t* scales,
                               cudaStream_t st, double lp = 0.0);
 cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st);
+// LayerNorm front-end, offline: l1gt = diag(gamma) (l1t hi + lo) as hi / lo rows,
+// cg = gamma^T L1', cb = beta^T L1' (float64 sums in fixed order).
+cudaError_t launch_ln_fold(const uint16_t* l1t, const float* gamma, const float* beta, int K,
+                           uint16_t* l1gt, float* cg, float* cb, cudaStream_t st);
 cudaError_t launch_gemm(const GemmParams& p, bool out_bf16, int num_sms, cudaStream_t st);
 int gemm_tile_n();
 

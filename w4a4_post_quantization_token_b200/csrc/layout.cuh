@@ -49,6 +49,20 @@ __host__ __device__ constexpr size_t qtab_bytes(int64_t K) {
   return static_cast<size_t>(K) * 2 + static_cast<size_t>(K / 32) * 16;
 }
 
+// LayerNorm table of the quantize kernel (shared-memory image, one bulk copy):
+//  * K/32 lines of 256 bytes, line b = gamma (bytes 0..127) and beta (128..255) of the 32
+//    values that block b of the transform input holds (for RPBH the gathered channels
+//    perm[32 b + j]), each half as 8 chunks of 16 bytes, chunk c stored at c ^ (b % 8);
+//  * RPBH only: K/32 lines of 128 bytes, gamma of channels 32 b .. 32 b + 31 in the same
+//    chunk order (the statistics pass reads the row unpermuted);
+//  * 16 bytes: mean_k beta_k as a float64, then 8 zero bytes.
+__host__ __device__ constexpr size_t ln_table_bytes(int64_t K, int kind) {
+  return static_cast<size_t>(K) * 8 + (kind == 2 ? static_cast<size_t>(K) * 4 : 0) + 16;
+}
+__host__ __device__ constexpr uint32_t ln_chunk_off(uint32_t b, uint32_t c) {
+  return 16u * (c ^ (b & 7u));
+}
+
 struct WeightsLayout {
   int64_t K = 0, N = 0, rank = 0, rp = 0, n_pad = 0;
   bool center = false;
@@ -62,10 +76,17 @@ struct WeightsLayout {
   size_t perm = 0;     // int32 [K]          RPBH gather indices
   size_t sgn = 0;      // f32   [K]          RPBH sign[k] / sqrt(32)
   size_t qtab = 0;     // uint8 [K*2 + K/32*16] RPBH table as the quantize kernel stages it
+  size_t lng = 0;      // f32   [K]          LayerNorm gamma (front-end on)
+  size_t lnb = 0;      // f32   [K]          LayerNorm beta
+  size_t lntab = 0;    // the quantize kernel's LayerNorm table, as it is staged in shared
+                       //   memory (ln_table_bytes)
+  size_t l1gt = 0;     // bf16  [kUCols, K]  diag(gamma) L1' as hi / lo rows (front-end, rank > 0)
+  size_t cg = 0;       // f32   [rp]         gamma^T L1'
+  size_t cb = 0;       // f32   [rp]         beta^T L1'
   size_t total = 0;
 
   __host__ __device__ static WeightsLayout make(int64_t K, int64_t N, int64_t rank, bool center,
-                                                int kind) {
+                                                int kind, bool ln = false) {
     WeightsLayout L;
     L.K = K; L.N = N; L.rank = rank; L.rp = rank > 0 ? kRankPad : 0; L.center = center;
     L.kind = kind;
@@ -82,6 +103,13 @@ struct WeightsLayout {
     L.perm = o;   o = align_up(o + (kind == 2 ? static_cast<size_t>(K) * 4 : 0), kAlign);
     L.sgn = o;    o = align_up(o + (kind == 2 ? static_cast<size_t>(K) * 4 : 0), kAlign);
     L.qtab = o;   o = align_up(o + (kind == 2 ? qtab_bytes(K) : 0), kAlign);
+    L.lng = o;    o = align_up(o + (ln ? static_cast<size_t>(K) * 4 : 0), kAlign);
+    L.lnb = o;    o = align_up(o + (ln ? static_cast<size_t>(K) * 4 : 0), kAlign);
+    L.lntab = o;  o = align_up(o + (ln ? ln_table_bytes(K, kind) : 0), kAlign);
+    const bool lr = ln && L.rp;
+    L.l1gt = o;   o = align_up(o + (lr ? static_cast<size_t>(kUCols) * K * 2 : 0), kAlign);
+    L.cg = o;     o = align_up(o + (lr ? static_cast<size_t>(L.rp) * 4 : 0), kAlign);
+    L.cb = o;     o = align_up(o + (lr ? static_cast<size_t>(L.rp) * 4 : 0), kAlign);
     L.total = o;
     return L;
   }
@@ -103,9 +131,11 @@ struct ActLayout {
   size_t sf = 0;       // uint8 tiled, rows padded to 128
   size_t mu = 0;       // f32 [m_pad]
   size_t u = 0;        // fp16 [M, rp]
+  size_t lnm = 0;      // f32 [m_pad] LayerNorm mean of x (front-end on)
+  size_t lnr = 0;      // f32 [m_pad] LayerNorm 1/sqrt(v + eps)
   size_t total = 0;
 
-  __host__ __device__ static ActLayout make(int64_t M, int64_t K, int64_t rank) {
+  __host__ __device__ static ActLayout make(int64_t M, int64_t K, int64_t rank, bool ln = false) {
     ActLayout L;
     L.M = M; L.K = K; L.rp = rank > 0 ? kRankPad : 0;
     L.m_pad = cdiv(M, 128) * 128;
@@ -115,6 +145,8 @@ struct ActLayout {
     L.sf = o;     o = align_up(o + sf_bytes(L.m_pad, K), kAlign);
     L.mu = o;     o = align_up(o + static_cast<size_t>(L.m_pad) * 4, kAlign);
     L.u = o;      o = align_up(o + static_cast<size_t>(M) * L.rp * 2, kAlign);
+    L.lnm = o;    o = align_up(o + (ln ? static_cast<size_t>(L.m_pad) * 4 : 0), kAlign);
+    L.lnr = o;    o = align_up(o + (ln ? static_cast<size_t>(L.m_pad) * 4 : 0), kAlign);
     L.total = o;
     return L;
   }

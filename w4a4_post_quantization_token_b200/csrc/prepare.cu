@@ -349,4 +349,43 @@ size_t prepare_syevd_lwork(int64_t K, int64_t N, int64_t rank) {
   return static_cast<size_t>(lwork);
 }
 
+// diag(gamma) L1' for the LayerNorm front-end; one block per low-rank column t.
+__global__ void k_ln_fold(const uint16_t* __restrict__ l1t, const float* __restrict__ gamma,
+                          const float* __restrict__ beta, int K, uint16_t* __restrict__ l1gt,
+                          float* __restrict__ cg, float* __restrict__ cb) {
+  const int t = blockIdx.x;
+  double sg = 0.0, sb = 0.0;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    const double v = bf16_bits_to_f64(l1t[static_cast<size_t>(t) * K + k]) +
+                     bf16_bits_to_f64(l1t[static_cast<size_t>(kRankPad + t) * K + k]);
+    const double vg = static_cast<double>(gamma[k]) * v;
+    const uint16_t hi = f64_to_bf16_bits(vg);
+    l1gt[static_cast<size_t>(t) * K + k] = hi;
+    l1gt[static_cast<size_t>(kRankPad + t) * K + k] = f64_to_bf16_bits(vg - bf16_bits_to_f64(hi));
+    sg += vg;
+    sb += static_cast<double>(beta[k]) * v;
+  }
+  __shared__ double rg[256], rb[256];
+  rg[threadIdx.x] = sg;
+  rb[threadIdx.x] = sb;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) {
+      rg[threadIdx.x] += rg[threadIdx.x + w];
+      rb[threadIdx.x] += rb[threadIdx.x + w];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    cg[t] = static_cast<float>(rg[0]);
+    cb[t] = static_cast<float>(rb[0]);
+  }
+}
+
+cudaError_t launch_ln_fold(const uint16_t* l1t, const float* gamma, const float* beta, int K,
+                           uint16_t* l1gt, float* cg, float* cb, cudaStream_t st) {
+  k_ln_fold<<<kRankPad, 256, 0, st>>>(l1t, gamma, beta, K, l1gt, cg, cb);
+  return cudaGetLastError();
+}
+
 }  // namespace kq

@@ -17,6 +17,11 @@
 //    X and of [L1'_hi; L1'_lo], the MMA accumulates 128 x 128 in TMEM, the epilogue forms
 //    hi + lo - mu c1 (mu from the quantize kernel) and stores fp16 (16-bit branch). For
 //    small M the K reduction is split over a cluster and reduced in distributed smem.
+//  * LayerNorm front-end (y = (x - m) rstd gamma + beta per token, ahead of the layer):
+//    the quantize kernel forms m, rstd and mean(y) from the staged row (a second, centred
+//    pass gives the variance) and normalises each block before centring it; the low-rank
+//    kernel still streams raw x, against diag(gamma) L1', and its epilogue applies
+//    y L1' = rstd (x diag(gamma) L1') - rstd m gamma^T L1' + beta^T L1'.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -116,11 +121,13 @@ __device__ __forceinline__ void encode_scaled2(const uint64_t (&v2)[16], float f
 
 // Transform + encode of one 32-element block (row r of the ring slot, block b). Writes the
 // codes (or, in debug mode, the transformed values) and returns the scale byte.
-template <int KIND, bool CENTER, bool DEBUG_XT>
+// CENTER: 0 off, 1 centring, 2 LayerNorm then centring of the normalised token.
+template <int KIND, int CENTER, bool DEBUG_XT>
 __device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const uint64_t (&Ap)[16],
                                                    const uint64_t (&Bp)[32], const uint8_t* rowb,
-                                                   const uint8_t* tables, int row, int b,
-                                                   float mu_hi, float mu_lo) {
+                                                   const uint8_t* tables, const uint8_t* lntab,
+                                                   int row, int b, float mu_hi, float mu_lo,
+                                                   float4 ln) {
   const float rs = 0.17677669529663687f;   // fp32(1 / sqrt(32))
   uint64_t v2[16];
   if (KIND == 2) {
@@ -162,6 +169,21 @@ __device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const u
     const uint64_t mh = f2pack(mu_hi, mu_hi), ml = f2pack(mu_lo, mu_lo);
 #pragma unroll
     for (int q = 0; q < 16; ++q) v2[q] = fsub2(fsub2(v2[q], mh), ml);
+  }
+  if (CENTER == 2) {
+    // y = (x - m) rstd gamma + beta, then y - mean(y) (ln = rstd, mean hi, mean lo)
+    const uint64_t rr = f2pack(ln.x, ln.x);
+    const uint64_t yh = f2pack(ln.y, ln.y), yl = f2pack(ln.z, ln.z);
+    const uint8_t* line = lntab + static_cast<uint32_t>(b) * 256u;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t o = ln_chunk_off(static_cast<uint32_t>(b), static_cast<uint32_t>(c));
+      const float4 g = *reinterpret_cast<const float4*>(line + o);
+      const float4 be = *reinterpret_cast<const float4*>(line + 128u + o);
+      v2[2 * c] = fsub2(fsub2(ffma2(fmul2(v2[2 * c], rr), f2pack(g.x, g.y), f2pack(be.x, be.y)), yh), yl);
+      v2[2 * c + 1] =
+          fsub2(fsub2(ffma2(fmul2(v2[2 * c + 1], rr), f2pack(g.z, g.w), f2pack(be.z, be.w)), yh), yl);
+    }
   }
   if (KIND == 1) kron_apply2(v2, Ap, Bp);
   if (KIND == 2) fwht32_2(v2);
@@ -243,7 +265,7 @@ __device__ __forceinline__ void store_scales(const QuantParams& p, bool valid, i
 // once per CTA, as one bulk copy of a table prepared with the weights; the Kronecker
 // factors live in registers. Centring: the warp forms each row's mean (fp32 block sums,
 // fp64 across blocks), then all u * K/32 blocks of the unit are spread over the lanes.
-template <int KIND, bool CENTER, bool DEBUG_XT>
+template <int KIND, int CENTER, bool DEBUG_XT>
 __global__ void __launch_bounds__(KIND == 1 ? 32 * kQMaxWarpsKron : 32 * kQMaxWarps, 1)
 k_quantize_rows(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -258,6 +280,8 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);             // [NW * S]
   uint64_t* tabbar = full + kQMaxWarps * kQMaxStages;
   float2* wmu = reinterpret_cast<float2*>(smem + kQMuOff) + 32 * warp;   // this warp's means
+  float4* wln = reinterpret_cast<float4*>(smem + kQLnOff) + 32 * warp;   // LayerNorm row terms
+  const uint8_t* lntab = smem + p.lntab_off;
   uint8_t* tables = smem + p.tables_off;
   uint8_t* wbufs = smem + p.bufs_off + static_cast<size_t>(warp) * S * slot_bytes;
   const int64_t units = cdiv(p.M, u);
@@ -296,9 +320,11 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
     fence_mbar_init();
     if (warp == 0) {
       prefetch_tmap(&p.tmap_x);
-      if (KIND == 2) {
-        mbar_arrive_expect_tx(tabbar, p.qtab_bytes);
-        bulk_load(tables, p.qtab, p.qtab_bytes, tabbar);
+      if (KIND == 2 || CENTER == 2) {
+        mbar_arrive_expect_tx(tabbar, (KIND == 2 ? p.qtab_bytes : 0u) +
+                                          (CENTER == 2 ? p.lntab_bytes : 0u));
+        if (KIND == 2) bulk_load(tables, p.qtab, p.qtab_bytes, tabbar);
+        if (CENTER == 2) bulk_load(smem + p.lntab_off, p.lntab, p.lntab_bytes, tabbar);
       }
     }
     for (int s = 0; s < S; ++s)
@@ -316,7 +342,8 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
   grid_dep_launch();                       // the low-rank / GEMM kernel may start its prologue
 
   bool ok = true;
-  if (KIND == 2) ok = __all_sync(0xffffffffu, mbar_wait(tabbar, 0, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
+  if (KIND == 2 || CENTER == 2)
+    ok = __all_sync(0xffffffffu, mbar_wait(tabbar, 0, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
   int64_t k = 0;
   for (int64_t l = warp; ok && l < nl; l += NW, ++k) {
     const int s = static_cast<int>(k % S);
@@ -344,7 +371,51 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
         const double mu64 = warp_sum_f64(part) / static_cast<double>(p.K);
         const float mu_hi = static_cast<float>(mu64);
         const float mu_lo = static_cast<float>(mu64 - static_cast<double>(mu_hi));
-        if (lane == 0) {
+        if (CENTER == 2) {
+          // second pass over the staged row, centred: sum d^2 and sum d gamma with
+          // d = (x - m_hi) - m_lo (fp32 per block, fp64 across blocks)
+          const uint64_t mh = f2pack(mu_hi, mu_hi), ml = f2pack(mu_lo, mu_lo);
+          const uint8_t* gbase = KIND == 2 ? lntab + static_cast<size_t>(p.K) * 8 : lntab;
+          const uint32_t gstride = KIND == 2 ? 128u : 256u;
+          double pv = 0.0, pg = 0.0;
+          for (int b = lane; b < nb; b += 32) {
+            uint64_t av = 0, ag = 0;
+            const uint8_t* gl = gbase + static_cast<uint32_t>(b) * gstride;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 q = *reinterpret_cast<const uint4*>(rowb + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
+              const float4 g0 = *reinterpret_cast<const float4*>(
+                  gl + ln_chunk_off(static_cast<uint32_t>(b), static_cast<uint32_t>(2 * c)));
+              const float4 g1 = *reinterpret_cast<const float4*>(
+                  gl + ln_chunk_off(static_cast<uint32_t>(b), static_cast<uint32_t>(2 * c + 1)));
+              const uint64_t d0 = fsub2(fsub2(bf16x2_to_f2(q.x), mh), ml);
+              const uint64_t d1 = fsub2(fsub2(bf16x2_to_f2(q.y), mh), ml);
+              const uint64_t d2 = fsub2(fsub2(bf16x2_to_f2(q.z), mh), ml);
+              const uint64_t d3 = fsub2(fsub2(bf16x2_to_f2(q.w), mh), ml);
+              av = ffma2(d0, d0, av); av = ffma2(d1, d1, av); av = ffma2(d2, d2, av); av = ffma2(d3, d3, av);
+              ag = ffma2(d0, f2pack(g0.x, g0.y), ag); ag = ffma2(d1, f2pack(g0.z, g0.w), ag);
+              ag = ffma2(d2, f2pack(g1.x, g1.y), ag); ag = ffma2(d3, f2pack(g1.z, g1.w), ag);
+            }
+            pv += static_cast<double>(f2lo(av)) + static_cast<double>(f2hi(av));
+            pg += static_cast<double>(f2lo(ag)) + static_cast<double>(f2hi(ag));
+          }
+          const double var = warp_sum_f64(pv) / static_cast<double>(p.K);
+          const double sdg = warp_sum_f64(pg);
+          const double rstd = 1.0 / sqrt(var + p.ln_eps);
+          const double mean_b = *reinterpret_cast<const double*>(lntab + p.lntab_bytes - 16u);
+          const double my = rstd * sdg / static_cast<double>(p.K) + mean_b;
+          const float my_hi = static_cast<float>(my);
+          const float my_lo = static_cast<float>(my - static_cast<double>(my_hi));
+          if (lane == 0) {
+            wmu[r] = make_float2(mu_hi, mu_lo);
+            wln[r] = make_float4(static_cast<float>(rstd), my_hi, my_lo, 0.f);
+            p.mu[row0 + r] = my_hi;
+            if (p.lnm != nullptr) {                  // null in the debug entry
+              p.lnm[row0 + r] = mu_hi;
+              p.lnr[row0 + r] = static_cast<float>(rstd);
+            }
+          }
+        } else if (lane == 0) {
           wmu[r] = make_float2(mu_hi, mu_lo);
           p.mu[row0 + r] = mu_hi;
         }
@@ -363,9 +434,12 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
       uint32_t sb = 0;
       if (valid) {
         float mh = 0.f, ml = 0.f;
+        float4 lr = make_float4(0.f, 0.f, 0.f, 0.f);
         if (CENTER) { const float2 m = wmu[r]; mh = m.x; ml = m.y; }
+        if (CENTER == 2) lr = wln[r];
         sb = quantize_block<KIND, CENTER, DEBUG_XT>(p, Ap, Bp, ub + static_cast<size_t>(r) * rstride,
-                                                    tables, static_cast<int>(row0 + r), b, mh, ml);
+                                                    tables, lntab, static_cast<int>(row0 + r), b, mh,
+                                                    ml, lr);
       }
       if (!DEBUG_XT) store_scales(p, valid, static_cast<int>(row0 + r), b, nb, nb_pad, sb);
       b += 32;
@@ -386,7 +460,10 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
     for (int i = blockIdx.x * nthr + tid; i < pad_rows * wpr; i += G * nthr) {
       const int rr = p.M + i / wpr, w = i % wpr;
       *reinterpret_cast<uint32_t*>(p.sf + sf_offset(rr, 4 * w, p.katoms)) = 0u;
-      if (w == 0) p.mu[rr] = 0.f;
+      if (w == 0) {
+        p.mu[rr] = 0.f;
+        if (CENTER == 2) { p.lnm[rr] = 0.f; p.lnr[rr] = 0.f; }
+      }
     }
   }
   // no TMA load may still be writing this CTA's shared memory when it exits: a warp
@@ -450,6 +527,22 @@ __device__ __forceinline__ uint32_t f2_to_half2_sat(float a, float b) {
   return *reinterpret_cast<const uint32_t*>(&h);
 }
 
+// One output of the U epilogue from the accumulated x L: acc - mu c1[j], or with the
+// LayerNorm front-end (L = diag(gamma) L1') rstd acc - rstd m cg[j] + cb[j] - mu c1[j],
+// which is y L1' - mean(y) c1 for y = LayerNorm(x).
+struct URowTerms { float mu, rs, rm; };
+__device__ __forceinline__ URowTerms u_row_terms(const LowRankParams& p, int row) {
+  URowTerms t;
+  t.mu = (p.mu != nullptr) ? p.mu[row] : 0.f;
+  t.rs = p.ln ? p.lnr[row] : 1.f;
+  t.rm = p.ln ? t.rs * p.lnm[row] : 0.f;
+  return t;
+}
+__device__ __forceinline__ float u_value(const LowRankParams& p, const URowTerms& t, float acc, int j) {
+  if (p.ln) return fmaf(t.rs, acc, fmaf(-t.rm, p.cg[j], p.cb[j])) - t.mu * p.c1[j];
+  return acc - t.mu * p.c1[j];
+}
+
 // Cluster reduction of the S fp32 partials ([64][128] column-major in each CTA's smem):
 // CTA ks finalises rows [ks*128/S, (ks+1)*128/S); S threads per row, 64/S columns each,
 // summed over the source CTAs in rank order.
@@ -472,11 +565,11 @@ __device__ __forceinline__ void lowrank_finish(const LowRankParams& p, const flo
     }
   }
   if (row < p.M) {
-    const float mu = (p.mu != nullptr) ? p.mu[row] : 0.f;
+    const URowTerms rt = u_row_terms(p, row);
     uint32_t* dst = reinterpret_cast<uint32_t*>(p.u + static_cast<size_t>(row) * kRankPad + j0);
 #pragma unroll
     for (int c = 0; c < kCols; c += 2)
-      dst[c / 2] = f2_to_half2_sat(acc[c] - mu * p.c1[j0 + c], acc[c + 1] - mu * p.c1[j0 + c + 1]);
+      dst[c / 2] = f2_to_half2_sat(u_value(p, rt, acc[c], j0 + c), u_value(p, rt, acc[c + 1], j0 + c + 1));
   }
 }
 
@@ -571,11 +664,11 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
     if (S == 1) {
       const int row = m0 + rl;
       if (ok && row < p.M) {
-        const float mu = (p.mu != nullptr) ? p.mu[row] : 0.f;
+        const URowTerms rt = u_row_terms(p, row);
         uint32_t packed[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          packed[j] = f2_to_half2_sat(u[2 * j] - mu * p.c1[2 * j], u[2 * j + 1] - mu * p.c1[2 * j + 1]);
+          packed[j] = f2_to_half2_sat(u_value(p, rt, u[2 * j], 2 * j), u_value(p, rt, u[2 * j + 1], 2 * j + 1));
         uint4* dst = reinterpret_cast<uint4*>(p.u + static_cast<size_t>(row) * kRankPad);
 #pragma unroll
         for (int v = 0; v < 8; ++v)
@@ -608,7 +701,7 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
 // ----------------------------------------------------------------------------------
 // host launchers
 // ----------------------------------------------------------------------------------
-template <int KIND, bool CENTER, bool DBG>
+template <int KIND, int CENTER, bool DBG>
 static cudaError_t launch_rows_t(const QuantParams& p, int num_sms, int block, size_t smem,
                                  cudaStream_t st) {
   auto fn = k_quantize_rows<KIND, CENTER, DBG>;
@@ -627,13 +720,13 @@ cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sm
                                  cudaStream_t st) {
   const int block = 32 * p.consumer_warps;
   const size_t smem = p.smem_bytes;
-  const int kind = p.kind, c = p.center ? 1 : 0;
+  const int kind = p.kind, c = p.center ? (p.ln ? 2 : 1) : 0;
 #define KQ_DISPATCH(KD, C)                                                             \
   if (kind == KD && c == C)                                                            \
-    return debug_xt ? launch_rows_t<KD, (C != 0), true>(p, num_sms, block, smem, st)   \
-                    : launch_rows_t<KD, (C != 0), false>(p, num_sms, block, smem, st);
-  KQ_DISPATCH(0, 0) KQ_DISPATCH(0, 1) KQ_DISPATCH(1, 0) KQ_DISPATCH(1, 1) KQ_DISPATCH(2, 0)
-  KQ_DISPATCH(2, 1) KQ_DISPATCH(3, 0)
+    return debug_xt ? launch_rows_t<KD, C, true>(p, num_sms, block, smem, st)          \
+                    : launch_rows_t<KD, C, false>(p, num_sms, block, smem, st);
+  KQ_DISPATCH(0, 0) KQ_DISPATCH(0, 1) KQ_DISPATCH(0, 2) KQ_DISPATCH(1, 0) KQ_DISPATCH(1, 1)
+  KQ_DISPATCH(1, 2) KQ_DISPATCH(2, 0) KQ_DISPATCH(2, 1) KQ_DISPATCH(2, 2) KQ_DISPATCH(3, 0)
 #undef KQ_DISPATCH
   return cudaErrorInvalidValue;
 }
