@@ -45,7 +45,8 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes + kSFABytes + kSFBBytes;
 constexpr uint32_t kEpiBuf = 4096;                       // 32 rows x 128 bytes
 constexpr int kEpiBufs = 2;                              // per epilogue warp
 constexpr uint32_t kEpiBytes = 4 * kEpiBufs * kEpiBuf;
-constexpr uint32_t kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes + 1024;
+constexpr uint32_t kColBytes = 4 * kBN * 4;              // per epilogue warp: s[n0 .. n0 + 191]
+constexpr uint32_t kSmemBytes = 1024 + kStages * kStageBytes + kEpiBytes + kColBytes + 1024;
 constexpr uint32_t kAccStride = kBN;                     // accumulators at columns 0, 192
 constexpr uint32_t kSFCol = 2 * kBN;                     // 384: one scale set per stage
 constexpr uint32_t kSFSetCols = 24;                      // SFA 8 columns, then SFB 16
@@ -83,6 +84,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
   uint8_t* stage0 = smem + 1024;
   uint8_t* epi0 = stage0 + kStages * kStageBytes;
+  float* col0 = reinterpret_cast<float*>(epi0 + kEpiBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int MT = static_cast<int>(cdiv(p.M, kBM));
@@ -263,6 +265,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
     grid_dep_wait();                       // mu comes from the quantize grid
     const int q = warp & 3;                               // TMEM lane quadrant
     uint8_t* stg = epi0 + static_cast<uint32_t>(q) * kEpiBufs * kEpiBuf;
+    float* scol = col0 + q * kBN;                          // this warp's copy of the tile's s
     const uint32_t r8 = static_cast<uint32_t>(lane & 7);
     int local = 0;
     uint32_t nstore = 0;
@@ -271,11 +274,23 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
       tile_coords(tile, MT, NT, mt, nt);
       const int m0 = mt * kBM, n0 = nt * kBN;
       const int buf = local & 1;
+      const int row = m0 + 32 * q + lane;
+      float mu = 0.f;
+      if (p.mu != nullptr) {
+        // the row's mean and the tile's 192 column sums, fetched while the MMAs run (the
+        // previous tile's reads of scol are done: same warp, in order)
+        mu = row < p.M ? p.mu[row] : 0.f;
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          const int n = n0 + 32 * c + lane;
+          scol[32 * c + lane] = n < p.N ? __ldg(p.s + n) : 0.f;
+        }
+        __syncwarp();
+      }
       const bool ok = __all_sync(0xffffffffu,
                                  mbar_wait(&acc_full[buf], (local >> 1) & 1, p.err, KQ_DEV_ERR_TIMEOUT_ACC));
       tc_fence_after();
-      const int row = m0 + 32 * q + lane;
-      const float mu = (p.mu != nullptr && row < p.M) ? p.mu[row] : 0.f;
       const uint32_t tbase = tmem + static_cast<uint32_t>(buf) * kAccStride +
                              (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
@@ -293,11 +308,10 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
         const int nc = n0 + 32 * c;
         float y[32];
         if (p.mu != nullptr) {
-          const int valid = min(32, p.N - nc);
-          const float4* s4 = reinterpret_cast<const float4*>(p.s + nc);
+          const float4* s4 = reinterpret_cast<const float4*>(scol + 32 * c);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const float4 sv = (4 * j < valid) ? __ldg(s4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 sv = s4[j];                       // same address in every lane
             y[4 * j + 0] = fmaf(mu, sv.x, __uint_as_float(r[4 * j + 0]));
             y[4 * j + 1] = fmaf(mu, sv.y, __uint_as_float(r[4 * j + 1]));
             y[4 * j + 2] = fmaf(mu, sv.z, __uint_as_float(r[4 * j + 2]));
