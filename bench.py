@@ -195,7 +195,8 @@ class Clocks:
                 "reasons": sorted(reasons), "samples": len(sms)}
 
 
-def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = None, ln=None):
+def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = None, ln=None,
+                        lut: bool = False):
     """Time the CPU oracle's online path (LayerNorm front-end when on, centre, transform,
     encode, fp64 contraction with both branches) on the first rows of the batch for about
     budget_s seconds."""
@@ -207,6 +208,11 @@ def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = No
         def linear(Xs, T, c, p):
             Y = oln.layernorm(Xs.double().numpy(), ln["gamma"], ln["beta"], ln["eps"])
             return olayer.linear(Y, T, c, p)
+    elif lut:
+        from oracle import lloydmax as olm
+
+        def linear(Xs, T, c, p):
+            return olm.linear(Xs.double().numpy(), T, c, p)
     else:
         linear = olayer.linear
     linear(X[:8], inp["T"], w.center, prep)                   # warm caches
@@ -283,6 +289,9 @@ def main():
                     help="skip the KroQuant-vs-SmoothQuant quantize-kernel timing")
     ap.add_argument("--center", action="store_true",
                     help="force per-token centring on (the workload's own setting otherwise)")
+    ap.add_argument("--codebook", choices=["mxfp4", "lloydmax"], default="mxfp4",
+                    help="activation format: MXFP4 (FP4 tensor cores) or the Lloyd-Max codebook "
+                         "with a per-token sigma (fp16 tensor cores; RPBH workloads)")
     ap.add_argument("--layernorm", action="store_true",
                     help="fuse a LayerNorm front-end (seeded gamma, beta) into the layer; "
                          "implies --center")
@@ -318,7 +327,8 @@ def main():
     if args.layernorm:
         from synthetic import make_layernorm
         ln = make_layernorm(w)
-    L = kq.Layer(w.K, w.N, w.rank, w.center, inp["T"], layernorm=ln)
+    L = kq.Layer(w.K, w.N, w.rank, w.center, inp["T"], layernorm=ln, codebook=args.codebook)
+    lut = args.codebook == "lloydmax"
     out_bf16 = args.out == "bf16"
     ydt = torch.bfloat16 if out_bf16 else torch.float32
     odt = kq.OUT_BF16 if out_bf16 else kq.OUT_F32
@@ -438,10 +448,16 @@ def main():
     M, K, N, rp = w.M, w.K, w.N, (64 if w.rank else 0)
     gemm_flops = 2.0 * M * N * K + 2.0 * M * N * w.rank + (M * N if w.center else 0)
     ybytes = M * N * (2 if out_bf16 else 4)
-    gemm_bytes = M * K / 2 + N * K / 2 + (M + N) * K / 32 + M * rp * 2 + N * rp * 2 + N * 4 + \
-        (M * 4 if w.center else 0) + ybytes
-    q_bytes = M * K * 2 + M * K / 2 + M * K / 32 + M * 4 + M * rp * 2
-    fp4_peak = peaks["bf16_sustained"] * FP4_OVER_BF16
+    if lut:   # fp16 operand and fp16 residual, no block scales
+        gemm_bytes = M * K * 2 + N * K * 2 + M * rp * 2 + N * rp * 2 + N * 4 + \
+            (M * 4 if w.center else 0) + ybytes
+        q_bytes = M * K * 2 + M * K * 2 + M * 8 + M * rp * 2
+    else:
+        gemm_bytes = M * K / 2 + N * K / 2 + (M + N) * K / 32 + M * rp * 2 + N * rp * 2 + N * 4 + \
+            (M * 4 if w.center else 0) + ybytes
+        q_bytes = M * K * 2 + M * K / 2 + M * K / 32 + M * 4 + M * rp * 2
+    # the contraction's own dtype: FP4 = 4 x the measured bf16 rate; fp16 = the bf16 rate
+    fp4_peak = peaks["bf16_sustained"] * (1.0 if lut else FP4_OVER_BF16)
     t_tensor = gemm_flops / (fp4_peak * 1e12)
     t_hbm = gemm_bytes / (peaks["hbm_gbs"] * 1e9)
     if g_ms >= q_ms:
@@ -458,7 +474,8 @@ def main():
         roof = {"kernel": "k_quantize_rows+k_lowrank_u", "bound": "hbm", "achieved": ach,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
     roof["traffic"] = measured_traffic(roof["kernel"], w.label)
-    roof["peak_source"] = peaks["source"] + (" (FP4 = 4 x sustained bf16)" if roof["unit"] == "TFLOP/s" else "")
+    roof["peak_source"] = peaks["source"] + (
+        (" (fp16 = sustained bf16)" if lut else " (FP4 = 4 x sustained bf16)") if roof["unit"] == "TFLOP/s" else "")
 
     # end-to-end through the host-buffer entry point (pinned memory, copies timed)
     e2e = None
@@ -488,7 +505,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import layer as olayer
         prep = olayer.prepare(inp["W"], inp["T"], w.rank)
-        v, rows, dt = oracle_tokens_per_s(w, inp, prep, budget_s=12.0, ln=ln)
+        v, rows, dt = oracle_tokens_per_s(w, inp, prep, budget_s=12.0, ln=ln, lut=lut)
         cpu = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"first {rows} of {w.M} tokens ({dt:.1f} s, fp64 NumPy, weights "
                          f"prepared beforehand)"}
@@ -501,11 +518,11 @@ def main():
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp16" if lut else "mxfp4",
         "data": "synthetic",
         "config": {"workload": w.label, "global_batch": w.M * world, "tokens_per_gpu": w.M,
                    "K": K, "N": N, "transform": w.transform, "center": w.center, "rank": w.rank,
-                   "layernorm": ln is not None, "out_dtype": args.out, "parallelism": f"replicas x{world} (token-sharded)",
+                   "layernorm": ln is not None, "codebook": args.codebook, "out_dtype": args.out, "parallelism": f"replicas x{world} (token-sharded)",
                    "l2": f"{R} rotating buffer sets of {set_bytes / 1e6:.0f} MB (> L2)",
                    "graph": graph is not None},
         "phases_ms": {"quantize": q_ms, "gemm": g_ms,

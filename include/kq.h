@@ -71,6 +71,21 @@ typedef enum {
 typedef enum { KQ_T_NONE = 0, KQ_T_KRON = 1, KQ_T_RPBH = 2 } kq_transform_kind;
 typedef enum { KQ_OUT_F32 = 0, KQ_OUT_BF16 = 1 } kq_out_dtype;
 
+/* Activation format.
+ *   KQ_CB_MXFP4: MXFP4 (OCP E2M1 elements, one E8M0 scale per 32 along K), contracted by
+ *     the block-scaled FP4 tensor-core MMA (KroQuant section 03).
+ *   KQ_CB_LLOYDMAX: OrbitQuant's single 16-level Lloyd-Max codebook of N(0, 1) for the
+ *     rotated coordinates (OrbitQuant section 03) with CentriQ's closed-form per-token
+ *     scale (abstract): sigma_m = RMS of the rotated (centred) token, each value the
+ *     level nearest to Xt / sigma_m (magnitude by midpoint thresholds, a magnitude on a
+ *     threshold taking the larger level; sign of Xt). The tensor cores have no codebook
+ *     format, so the decoded operand fp16(fp32(sigma_m) * fp32(level)) is stored and the
+ *     weights' MXFP4 residual is decoded to fp16 offline: the contraction is an fp16
+ *     tensor-core GEMM (a quarter of the FP4 rate, four times the operand bytes). Needs
+ *     the RPBH transform (whose coordinates the codebook is designed for) or none, and
+ *     no LayerNorm front-end. */
+typedef enum { KQ_CB_MXFP4 = 0, KQ_CB_LLOYDMAX = 1 } kq_act_format;
+
 /* The online block transform P (KroQuant section 02; OrbitQuant section 03).
  * All pointers are HOST memory, read during the call.
  *   KQ_T_KRON: P = blockdiag(A (x) B) over the K/32 blocks, A a_dim x a_dim and
@@ -116,6 +131,7 @@ typedef struct {
   int32_t center;        /* 1: per-token mean centring with rank-1 restore (CentriQ) */
   kq_transform_desc t;
   kq_layernorm_desc ln;  /* zero-initialised: no front-end */
+  int32_t codebook;      /* kq_act_format; 0 (MXFP4) when zero-initialised */
 } kq_layer_desc;
 
 /* ---------------------------------------------------------------------------------
@@ -253,15 +269,23 @@ kq_status kq_weights_unpack(const kq_layer_desc *desc, const void *weights, void
                             kq_stream_t stream);
 
 /* Fill an activation workspace from canonical parts (mu may be null when centring is
- * off; U_f16, the low-rank activations as fp16 [M, rank], may be null when rank == 0). */
+ * off; U_f16, the low-rank activations as fp16 [M, rank], may be null when rank == 0).
+ * For a KQ_CB_LLOYDMAX layer, codes is the fp16 operand [M, K] and scales the fp32
+ * per-token sigma [M]. */
 kq_status kq_act_pack(const kq_layer_desc *desc, const void *codes, const void *scales,
                       const float *mu, const void *U_f16, int32_t M, void *act,
                       size_t act_bytes, kq_stream_t stream);
 
 /* Read an activation workspace back into canonical parts (null pointers skip).
- * U_f16 receives fp16 [M, rank]. */
+ * U_f16 receives fp16 [M, rank]. For a KQ_CB_LLOYDMAX layer, codes receives the fp16
+ * operand [M, K] and scales the fp32 per-token sigma [M]. */
 kq_status kq_act_unpack(const kq_layer_desc *desc, const void *act, int32_t M, void *codes,
                         void *scales, float *mu, void *U_f16, kq_stream_t stream);
+
+/* The library's 16-level Lloyd-Max codebook of N(0, 1) (host memory, no device work):
+ * levels8 = the 8 positive levels ascending, thresholds7 = the midpoints between them,
+ * computed once by Lloyd's alternation in float64. Either pointer may be null. */
+kq_status kq_lloydmax_codebook(double *levels8, double *thresholds7);
 
 /* ---------------------------------------------------------------------------------
  * Debug entry points (each runs one stage of the online half in isolation).

@@ -34,8 +34,8 @@ def test_library_is_in_tree_and_versioned():
 def test_struct_layout_matches_c():
     # kq_transform_desc: int32 + ptr + int32 + ptr + int32 + ptr + ptr (with padding) = 56
     assert ctypes.sizeof(kq._TransformDesc) == 56
-    # + kq_layernorm_desc: int32 + float + ptr + ptr = 24
-    assert ctypes.sizeof(kq._LayerDesc) == 16 + 56 + 24
+    # + kq_layernorm_desc: int32 + float + ptr + ptr = 24, + int32 codebook (padded to 8)
+    assert ctypes.sizeof(kq._LayerDesc) == 16 + 56 + 24 + 8
 
 
 def _kron():
@@ -144,3 +144,36 @@ def test_layernorm_descriptor_validation():
     # the SmoothQuant comparator has no front-end
     L0 = kq.Layer(K, N, 0, True, {"kind": "none"}, layernorm=_ln(K))
     assert kq.lib.kq_smooth_quantize_act(L0.desc, ok, ok, 8, ok, 1 << 20, None) == 1
+
+
+def _rpbh(K):
+    return {"kind": "rpbh", "perm": np.arange(K)[::-1].copy(), "sign": np.ones(K, np.int8)}
+
+
+def test_codebook_descriptor_validation():
+    K, N = 256, 128
+    plain = kq.Layer(K, N, 16, True, _rpbh(K))
+    lut = kq.Layer(K, N, 16, True, _rpbh(K), codebook="lloydmax")
+    # the decoded fp16 residual rides along with the weights; the activation operand is
+    # fp16 (2 bytes per element) with one sigma per token and no block scales
+    assert kq.weights_bytes(lut) >= kq.weights_bytes(plain) + N * K * 2
+    assert kq.act_bytes(lut, 300) >= 300 * K * 2 + 384 * 4
+    assert kq.weights_bytes(kq.Layer(K, N, 0, False, {"kind": "none"}, codebook="lloydmax")) > 0
+    # designed for the RPBH coordinates: not with the Kronecker transform, not behind the
+    # LayerNorm front-end
+    assert kq.weights_bytes(kq.Layer(K, N, 16, True, _kron(), codebook="lloydmax")) == 0
+    ln = {"gamma": np.ones(K, np.float32), "beta": np.zeros(K, np.float32), "eps": 1e-6}
+    assert kq.weights_bytes(kq.Layer(K, N, 16, True, _rpbh(K), layernorm=ln, codebook="lloydmax")) == 0
+    bad = kq.Layer(K, N, 16, True, _rpbh(K))
+    bad._desc.codebook = 2
+    assert kq.weights_bytes(bad) == 0
+
+
+def test_library_codebook_matches_the_oracle():
+    """The library computes its Lloyd-Max codebook with its own host code; it must be the
+    oracle's fixed point to float64 rounding."""
+    from oracle import lloydmax as lm
+    lv, th = kq.lloydmax_codebook()
+    pos, pth = lm.magnitudes()
+    np.testing.assert_allclose(lv, pos, rtol=1e-13, atol=0)
+    np.testing.assert_allclose(th, pth, rtol=1e-13, atol=0)

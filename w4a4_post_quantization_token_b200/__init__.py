@@ -15,7 +15,7 @@ import numpy as np
 
 __all__ = ["KQError", "Layer", "lib", "library_path", "weights_bytes", "act_bytes",
            "prepare_ws_bytes", "prepare_weights", "prepare_weights_lp", "debug_encode_lp_f32", "quantize_act", "smooth_quantize_act", "linear",
-           "linear_noalloc",
+           "linear_noalloc", "lloydmax_codebook", "CB_MXFP4", "CB_LLOYDMAX",
            "linear_host", "NOALLOC_WORKSPACE_BYTES",
            "gemm", "weights_pack", "weights_unpack", "act_pack", "act_unpack",
            "debug_transform", "debug_encode_f32", "last_device_error", "status_string",
@@ -24,6 +24,8 @@ __all__ = ["KQError", "Layer", "lib", "library_path", "weights_bytes", "act_byte
 OUT_F32, OUT_BF16 = 0, 1
 T_NONE, T_KRON, T_RPBH = 0, 1, 2
 _KIND = {"none": T_NONE, "kron": T_KRON, "rpbh": T_RPBH}
+CB_MXFP4, CB_LLOYDMAX = 0, 1
+_CODEBOOK = {"mxfp4": CB_MXFP4, "lloydmax": CB_LLOYDMAX}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libkq.so")
@@ -34,7 +36,7 @@ SYMBOLS = ["kq_weights_bytes", "kq_act_bytes", "kq_prepare_ws_bytes", "kq_prepar
            "kq_weights_unpack", "kq_act_pack", "kq_act_unpack", "kq_debug_transform",
            "kq_debug_encode_f32", "kq_last_device_error", "kq_status_string", "kq_version",
            "kq_linear_noalloc", "kq_smooth_quantize_act", "kq_prepare_weights_lp",
-           "kq_debug_encode_lp_f32"]
+           "kq_debug_encode_lp_f32", "kq_lloydmax_codebook"]
 
 
 class KQError(RuntimeError):
@@ -63,7 +65,8 @@ class _LayerNormDesc(ctypes.Structure):
 
 class _LayerDesc(ctypes.Structure):
     _fields_ = [("K", ctypes.c_int32), ("N", ctypes.c_int32), ("rank", ctypes.c_int32),
-                ("center", ctypes.c_int32), ("t", _TransformDesc), ("ln", _LayerNormDesc)]
+                ("center", ctypes.c_int32), ("t", _TransformDesc), ("ln", _LayerNormDesc),
+                ("codebook", ctypes.c_int32)]
 
 
 _P = ctypes.c_void_p
@@ -91,6 +94,7 @@ _sigs = {
     "kq_debug_transform": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, _P, _P]),
     "kq_debug_encode_f32": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P, _P]),
     "kq_last_device_error": (ctypes.c_int, [_D, _P, ctypes.c_int32, _P]),
+    "kq_lloydmax_codebook": (ctypes.c_int, [_P, _P]),
     "kq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kq_version": (ctypes.c_char_p, []),
 }
@@ -98,6 +102,15 @@ for _name, (_res, _args) in _sigs.items():
     _f = getattr(lib, _name)
     _f.restype = _res
     _f.argtypes = _args
+
+
+def lloydmax_codebook() -> tuple[np.ndarray, np.ndarray]:
+    """The library's (8 positive levels, 7 thresholds) of its 16-level Lloyd-Max codebook."""
+    lv = np.zeros(8, np.float64)
+    th = np.zeros(7, np.float64)
+    _check(lib.kq_lloydmax_codebook(lv.ctypes.data_as(_P), th.ctypes.data_as(_P)),
+           "kq_lloydmax_codebook")
+    return lv, th
 
 
 def status_string(s: int) -> str:
@@ -116,10 +129,13 @@ class Layer:
     ``{"kind": "rpbh", "perm": int[K], "sign": +-1[K]}`` or ``{"kind": "none"}``.
     ``layernorm`` (optional) is ``{"gamma": float[K], "beta": float[K], "eps": float}``: the
     fused LayerNorm front-end (needs ``center``).
+    ``codebook`` is ``"mxfp4"`` (default) or ``"lloydmax"``: the 16-level Lloyd-Max
+    codebook with a per-token sigma (RPBH or no transform; activations reach the fp16
+    tensor-core GEMM as decoded fp16 values).
     The host arrays are kept alive by this object."""
 
     def __init__(self, K: int, N: int, rank: int, center: bool, transform: dict,
-                 layernorm: dict | None = None):
+                 layernorm: dict | None = None, codebook: str = "mxfp4"):
         self.K, self.N, self.rank, self.center = int(K), int(N), int(rank), bool(center)
         self.transform = transform
         kind = _KIND[transform["kind"]]
@@ -147,8 +163,9 @@ class Layer:
             ln.on, ln.eps = 1, float(layernorm.get("eps", 1e-6))
             ln.gamma = g.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
             ln.beta = b.ctypes.data_as(ctypes.POINTER(ctypes.c_float))
+        self.codebook = codebook
         self._desc = _LayerDesc(K=self.K, N=self.N, rank=self.rank, center=int(self.center), t=t,
-                                ln=ln)
+                                ln=ln, codebook=_CODEBOOK[codebook])
 
     @property
     def desc(self):

@@ -99,6 +99,10 @@ kq_status check_desc(const kq_layer_desc* d) {
     }
     default: return KQ_ERR_INVALID_ARG;
   }
+  if (d->codebook != KQ_CB_MXFP4 && d->codebook != KQ_CB_LLOYDMAX) return KQ_ERR_INVALID_ARG;
+  // the codebook is designed for the Gaussian coordinates of the RPBH rotation
+  if (d->codebook == KQ_CB_LLOYDMAX && (d->t.kind == KQ_T_KRON || d->ln.on != 0))
+    return KQ_ERR_INVALID_ARG;
   if (d->ln.on != 0) {
     // the front-end normalises, then the layer centres the normalised token (CentriQ)
     if (d->ln.on != 1 || d->center != 1) return KQ_ERR_INVALID_ARG;
@@ -117,10 +121,11 @@ kq_status check_ln_values(const kq_layer_desc* d) {
 }
 
 WeightsLayout wlayout(const kq_layer_desc* d) {
-  return WeightsLayout::make(d->K, d->N, d->rank, d->center != 0, d->t.kind, d->ln.on != 0);
+  return WeightsLayout::make(d->K, d->N, d->rank, d->center != 0, d->t.kind, d->ln.on != 0,
+                             d->codebook == KQ_CB_LLOYDMAX);
 }
 ActLayout alayout(const kq_layer_desc* d, int M) {
-  return ActLayout::make(M, d->K, d->rank, d->ln.on != 0);
+  return ActLayout::make(M, d->K, d->rank, d->ln.on != 0, d->codebook == KQ_CB_LLOYDMAX);
 }
 
 // LayerNorm table image (layout: ln_table_bytes). Position j of block b holds channel
@@ -169,6 +174,49 @@ kq_status write_ln_weights(const kq_layer_desc* d, uint8_t* w, cudaStream_t st) 
     return KQ_ERR_CUDA;
   if (cudaStreamSynchronize(st) != cudaSuccess) return KQ_ERR_CUDA;   // host table
   return KQ_OK;
+}
+
+// 16-level Lloyd-Max quantizer of N(0, 1): Lloyd's alternation of the two optimality
+// conditions (thresholds at the midpoints of neighbouring levels; each level the mean of
+// N(0, 1) over its cell, (pdf(a) - pdf(b)) / (cdf(b) - cdf(a))), in float64 from a uniform
+// start, the levels kept symmetric about 0, until a sweep moves no level by more than
+// 1e-15. Computed once; the 8 positive levels and the 7 thresholds between them.
+struct LloydMax { double mag[8]; double thr[7]; };
+const LloydMax& lloyd_max16() {
+  static LloydMax lm;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    constexpr int n = 16;
+    const double inv_sqrt_2pi = 0.3989422804014327;
+    auto pdf = [&](double x) { return inv_sqrt_2pi * std::exp(-0.5 * x * x); };
+    auto cdf = [](double x) { return 0.5 * std::erfc(-x / std::sqrt(2.0)); };
+    double lv[n], nx[n];
+    for (int i = 0; i < n; ++i) lv[i] = -2.0 + 4.0 * i / (n - 1);
+    for (int it = 0; it < 200000; ++it) {
+      double move = 0.0;
+      for (int i = 0; i < n; ++i) {
+        const bool lo_inf = i == 0, hi_inf = i == n - 1;
+        const double a = lo_inf ? 0.0 : 0.5 * (lv[i - 1] + lv[i]);
+        const double b = hi_inf ? 0.0 : 0.5 * (lv[i] + lv[i + 1]);
+        const double pa = lo_inf ? 0.0 : pdf(a), pb = hi_inf ? 0.0 : pdf(b);
+        const double ca = lo_inf ? 0.0 : cdf(a), cb = hi_inf ? 1.0 : cdf(b);
+        nx[i] = (pa - pb) / (cb - ca);
+      }
+      for (int i = 0; i < n / 2; ++i) {
+        const double v = 0.5 * (nx[n - 1 - i] - nx[i]);
+        nx[i] = -v;
+        nx[n - 1 - i] = v;
+      }
+      for (int i = 0; i < n; ++i) {
+        move = std::fmax(move, std::fabs(nx[i] - lv[i]));
+        lv[i] = nx[i];
+      }
+      if (move < 1e-15) break;
+    }
+    for (int i = 0; i < 8; ++i) lm.mag[i] = lv[8 + i];
+    for (int i = 0; i < 7; ++i) lm.thr[i] = 0.5 * (lm.mag[i] + lm.mag[i + 1]);
+  });
+  return lm;
 }
 
 // Gauss-Jordan inverse with partial pivoting (float64); false if singular.
@@ -297,8 +345,15 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
                  CU_TENSOR_MAP_SWIZZLE_64B))
     return KQ_ERR_CUDA;
   const bool ln = d->ln.on != 0;
-  if (ln && inv_s) return KQ_ERR_INVALID_ARG;
-  p->tables_off = ln ? kQTablesMinLn : kQTablesMin;
+  const bool lut = d->codebook == KQ_CB_LLOYDMAX;
+  if ((ln || lut) && inv_s) return KQ_ERR_INVALID_ARG;
+  p->tables_off = (ln || lut) ? kQTablesMinLn : kQTablesMin;
+  if (lut) {
+    const LloydMax& cb = lloyd_max16();
+    p->lut = 1;
+    for (int i = 0; i < 8; ++i) p->lut_mag[i] = static_cast<float>(cb.mag[i]);
+    for (int i = 0; i < 7; ++i) p->lut_thr[i] = static_cast<float>(cb.thr[i]);
+  }
   p->qtab_bytes = d->t.kind == KQ_T_RPBH ? static_cast<uint32_t>(qtab_bytes(K)) : 0u;
   const size_t table_bytes = inv_s ? static_cast<size_t>(K) * 4 : p->qtab_bytes;
   size_t tables_end = p->tables_off + table_bytes;
@@ -342,6 +397,12 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
     if (ln) {
       p->lnm = reinterpret_cast<float*>(act + AL.lnm);
       p->lnr = reinterpret_cast<float*>(act + AL.lnr);
+    }
+    if (lut) {
+      p->a16 = reinterpret_cast<uint16_t*>(act + AL.codes);
+      p->sig = reinterpret_cast<float*>(act + AL.sig);
+      p->codes = nullptr;
+      p->sf = nullptr;
     }
   }
   p->qtab = weights ? static_cast<const uint8_t*>(weights) + WL.qtab : nullptr;
@@ -397,14 +458,27 @@ kq_status run_gemm(const kq_layer_desc* d, const void* weights, const uint8_t* a
   const bool bf16 = out_dtype == KQ_OUT_BF16;
   GemmParams gp;
   std::memset(&gp, 0, sizeof(gp));
-  if (!make_tmap(&gp.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, act + AL.codes, static_cast<uint64_t>(K / 2),
-                 static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), 128, 128,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
-    return KQ_ERR_CUDA;
-  if (!make_tmap(&gp.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w + WL.rcodes, static_cast<uint64_t>(K / 2),
-                 static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), 128, bn,
-                 CU_TENSOR_MAP_SWIZZLE_128B))
-    return KQ_ERR_CUDA;
+  if (d->codebook == KQ_CB_LLOYDMAX) {
+    // fp16 operand [M, K] and fp16 residual [N, K], 64-element (128-byte) k-tiles
+    gp.f16 = 1;
+    if (!make_tmap(&gp.tmap_a, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, act + AL.codes, static_cast<uint64_t>(K),
+                   static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, 64, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return KQ_ERR_CUDA;
+    if (!make_tmap(&gp.tmap_b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w + WL.rf16, static_cast<uint64_t>(K),
+                   static_cast<uint64_t>(N), static_cast<uint64_t>(K) * 2, 64, bn,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return KQ_ERR_CUDA;
+  } else {
+    if (!make_tmap(&gp.tmap_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, act + AL.codes, static_cast<uint64_t>(K / 2),
+                   static_cast<uint64_t>(M), static_cast<uint64_t>(K / 2), 128, 128,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return KQ_ERR_CUDA;
+    if (!make_tmap(&gp.tmap_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, w + WL.rcodes, static_cast<uint64_t>(K / 2),
+                   static_cast<uint64_t>(N), static_cast<uint64_t>(K / 2), 128, bn,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return KQ_ERR_CUDA;
+  }
   // low-rank step: only the first 32 of the 64 stored columns when rank <= 32 (the rest
   // are zero), as 64-byte rows with the 64-byte swizzle
   const int lrk = d->rank == 0 ? 0 : (d->rank <= 32 ? 32 : kRankPad);
@@ -485,6 +559,10 @@ kq_status prepare_weights_impl(const kq_layer_desc* desc, const void* W_bf16, vo
         cudaStreamSynchronize(a.stream) != cudaSuccess)
       return KQ_ERR_CUDA;
   }
+  if (desc->codebook == KQ_CB_LLOYDMAX &&
+      (decode_residual_f16(wlayout(desc), static_cast<uint8_t*>(weights), a.stream) != cudaSuccess ||
+       cudaStreamSynchronize(a.stream) != cudaSuccess))
+    return KQ_ERR_CUDA;
   return write_ln_weights(desc, static_cast<uint8_t*>(weights), a.stream);
 }
 
@@ -505,6 +583,13 @@ const char* kq_status_string(kq_status s) {
     case KQ_ERR_NO_SM100: return "device is not sm_100 (B200)";
   }
   return "unknown status";
+}
+
+kq_status kq_lloydmax_codebook(double* levels8, double* thresholds7) {
+  const LloydMax& cb = lloyd_max16();
+  if (levels8) for (int i = 0; i < 8; ++i) levels8[i] = cb.mag[i];
+  if (thresholds7) for (int i = 0; i < 7; ++i) thresholds7[i] = cb.thr[i];
+  return KQ_OK;
 }
 
 const char* kq_version(void) { return "kq 0.1 (sm_100a, tcgen05 mxf4)"; }
@@ -557,7 +642,8 @@ kq_status kq_smooth_quantize_act(const kq_layer_desc* desc, const float* inv_s,
                                  kq_stream_t stream) {
   kq_status s = check_desc(desc);
   if (s != KQ_OK) return s;
-  if (desc->t.kind != KQ_T_NONE || desc->center || desc->rank != 0 || desc->ln.on)
+  if (desc->t.kind != KQ_T_NONE || desc->center || desc->rank != 0 || desc->ln.on ||
+      desc->codebook != KQ_CB_MXFP4)
     return KQ_ERR_INVALID_ARG;
   if (M <= 0 || !inv_s || !X_bf16 || !act) return KQ_ERR_INVALID_ARG;
   if (!aligned(inv_s) || !aligned(X_bf16) || !aligned(act)) return KQ_ERR_ALIGNMENT;
@@ -649,6 +735,8 @@ kq_status kq_weights_pack(const kq_layer_desc* desc, const void* r_codes, const 
       return KQ_ERR_CUDA;
     if (cudaStreamSynchronize(st) != cudaSuccess) return KQ_ERR_CUDA;   // host locals
   }
+  if (desc->codebook == KQ_CB_LLOYDMAX && decode_residual_f16(WL, w, st) != cudaSuccess)
+    return KQ_ERR_CUDA;
   return write_ln_weights(desc, w, st);
 }
 

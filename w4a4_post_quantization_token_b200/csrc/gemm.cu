@@ -71,7 +71,10 @@ __device__ __forceinline__ void tile_coords(int tile, int MT, int NT, int& mt, i
   nt = r / gm;
 }
 
-template <bool OUT_BF16>
+// F16: the main loop contracts fp16 operands (Lloyd-Max activations decoded to fp16 and
+// the residual decoded to fp16) with kind::f16 MMAs, 64 elements (128 bytes) per k-tile;
+// the scale copier then only relays the stage barriers.
+template <bool OUT_BF16, bool F16>
 __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_constant__ GemmParams p) {
   using namespace gemm;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -90,7 +93,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
   const int MT = static_cast<int>(cdiv(p.M, kBM));
   const int NT = static_cast<int>(cdiv(p.N, kBN));
   const int T = MT * NT;
-  const int KT = static_cast<int>(cdiv(p.K, kTileK));
+  const int KT = static_cast<int>(cdiv(p.K, F16 ? 64 : kTileK));
   const bool lowrank = p.rank_pad > 0;
   const int steps = KT + (lowrank ? 1 : 0);
 
@@ -136,7 +139,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
           }
           uint8_t* a = stage0 + s * kStageBytes;
           uint8_t* b = a + kABytes;
-          if (ks < KT) {
+          if (ks < KT && F16) {
+            mbar_arrive_expect_tx(&full[s], kABytes + kBBytes);
+            tma_load_2d(a, &p.tmap_a, ks * 64, m0, &full[s]);
+            tma_load_2d(b, &p.tmap_b, ks * 64, n0, &full[s]);
+          } else if (ks < KT) {
             uint8_t* sfa = b + kBBytes;
             uint8_t* sfb = sfa + kSFABytes;
             mbar_arrive_expect_tx(&full[s], kStageBytes);
@@ -191,7 +198,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
           tc_fence_after();
           const uint64_t so = static_cast<uint64_t>(s) * kStageDesc;
           const uint64_t ad = adesc0 + so, bd = bdesc0 + so;
-          if (ks < KT) {
+          if (ks < KT && F16) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              mma_bf16(d, ad + 2 * kk, bd + 2 * kk, idf16, (ks > 0 || kk > 0) ? 1u : 0u);
+          } else if (ks < KT) {
             const uint32_t fa = tmem + kSFCol + static_cast<uint32_t>(s) * kSFSetCols;
             const uint32_t fb = fa + 8 + shift;
             const uint32_t acc0 = ks > 0 ? 1u : 0u;
@@ -244,7 +255,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
             break;
           }
           tc_fence_after();
-          if (ks < KT) {
+          if (ks < KT && !F16) {
             const uint32_t fa = tmem + kSFCol + static_cast<uint32_t>(s) * kSFSetCols;
             const uint32_t fb = fa + 8;
             const uint64_t sd = sdesc0 + static_cast<uint64_t>(s) * kStageDesc;
@@ -376,7 +387,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
 
 template <bool BF16>
 static cudaError_t launch_gemm_t(const GemmParams& p, int num_sms, cudaStream_t st) {
-  auto fn = k_gemm_mxf4<BF16>;
+  auto fn = p.f16 ? k_gemm_mxf4<BF16, true> : k_gemm_mxf4<BF16, false>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(gemm::kSmemBytes));
   if (e != cudaSuccess) return e;

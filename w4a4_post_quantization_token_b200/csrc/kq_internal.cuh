@@ -51,6 +51,11 @@ struct QuantParams {
   uint32_t lntab_off;          // its shared-memory offset (128-byte aligned)
   float* lnm;                  // out: per-token mean of x [m_pad]
   float* lnr;                  // out: per-token 1/sqrt(v + eps) [m_pad]
+  int lut;                     // Lloyd-Max activations: fp16 operand out, no block scales
+  float lut_mag[8];            //   positive codebook levels (ascending)
+  float lut_thr[7];            //   thresholds between them
+  uint16_t* a16;               // out: fp16 operand [M, K]
+  float* sig;                  // out: per-token sigma [m_pad]
   float* xt;                   // debug: transformed values [M, K] (debug launch only)
   uint32_t* err;
 };
@@ -83,6 +88,8 @@ struct GemmParams {
   void* y;                     // [M, N] f32 or bf16
   int M, N, K;
   int rank_pad;                // low-rank K of the GEMM: 0, 32 (64-byte swizzle) or 64 (128-byte)
+  int f16;                     // 1: the main loop is fp16 x fp16 (Lloyd-Max operand, decoded
+                               //    residual), tmap_a / tmap_b are fp16 [M|N, K], no scales
   int64_t katoms;
   uint32_t* err;
 };

@@ -83,10 +83,11 @@ struct WeightsLayout {
   size_t l1gt = 0;     // bf16  [kUCols, K]  diag(gamma) L1' as hi / lo rows (front-end, rank > 0)
   size_t cg = 0;       // f32   [rp]         gamma^T L1'
   size_t cb = 0;       // f32   [rp]         beta^T L1'
+  size_t rf16 = 0;     // fp16  [N, K]       residual decoded to fp16 (Lloyd-Max activations)
   size_t total = 0;
 
   __host__ __device__ static WeightsLayout make(int64_t K, int64_t N, int64_t rank, bool center,
-                                                int kind, bool ln = false) {
+                                                int kind, bool ln = false, bool lut = false) {
     WeightsLayout L;
     L.K = K; L.N = N; L.rank = rank; L.rp = rank > 0 ? kRankPad : 0; L.center = center;
     L.kind = kind;
@@ -110,6 +111,7 @@ struct WeightsLayout {
     L.l1gt = o;   o = align_up(o + (lr ? static_cast<size_t>(kUCols) * K * 2 : 0), kAlign);
     L.cg = o;     o = align_up(o + (lr ? static_cast<size_t>(L.rp) * 4 : 0), kAlign);
     L.cb = o;     o = align_up(o + (lr ? static_cast<size_t>(L.rp) * 4 : 0), kAlign);
+    L.rf16 = o;   o = align_up(o + (lut ? static_cast<size_t>(N) * K * 2 : 0), kAlign);
     L.total = o;
     return L;
   }
@@ -126,27 +128,31 @@ __host__ __device__ constexpr int u_split(int64_t M, int64_t K) {
 
 struct ActLayout {
   int64_t M = 0, m_pad = 0, K = 0, rp = 0;
+  bool lut = false;    // Lloyd-Max activations: codes holds the fp16 operand, no sf
   size_t err = 0;      // uint32 device error word
-  size_t codes = 0;    // uint8 [M, K/2]
-  size_t sf = 0;       // uint8 tiled, rows padded to 128
+  size_t codes = 0;    // uint8 [M, K/2] (MXFP4) or fp16 [M, K] (Lloyd-Max operand)
+  size_t sf = 0;       // uint8 tiled, rows padded to 128 (MXFP4 only)
   size_t mu = 0;       // f32 [m_pad]
   size_t u = 0;        // fp16 [M, rp]
   size_t lnm = 0;      // f32 [m_pad] LayerNorm mean of x (front-end on)
   size_t lnr = 0;      // f32 [m_pad] LayerNorm 1/sqrt(v + eps)
+  size_t sig = 0;      // f32 [m_pad] per-token sigma (Lloyd-Max activations)
   size_t total = 0;
 
-  __host__ __device__ static ActLayout make(int64_t M, int64_t K, int64_t rank, bool ln = false) {
+  __host__ __device__ static ActLayout make(int64_t M, int64_t K, int64_t rank, bool ln = false,
+                                            bool lut = false) {
     ActLayout L;
-    L.M = M; L.K = K; L.rp = rank > 0 ? kRankPad : 0;
+    L.M = M; L.K = K; L.rp = rank > 0 ? kRankPad : 0; L.lut = lut;
     L.m_pad = cdiv(M, 128) * 128;
     size_t o = 0;
     L.err = o;    o = kHdrBytes;
-    L.codes = o;  o = align_up(o + static_cast<size_t>(M) * (K / 2), kAlign);
-    L.sf = o;     o = align_up(o + sf_bytes(L.m_pad, K), kAlign);
+    L.codes = o;  o = align_up(o + static_cast<size_t>(M) * (lut ? K * 2 : K / 2), kAlign);
+    L.sf = o;     o = align_up(o + (lut ? 0 : sf_bytes(L.m_pad, K)), kAlign);
     L.mu = o;     o = align_up(o + static_cast<size_t>(L.m_pad) * 4, kAlign);
     L.u = o;      o = align_up(o + static_cast<size_t>(M) * L.rp * 2, kAlign);
     L.lnm = o;    o = align_up(o + (ln ? static_cast<size_t>(L.m_pad) * 4 : 0), kAlign);
     L.lnr = o;    o = align_up(o + (ln ? static_cast<size_t>(L.m_pad) * 4 : 0), kAlign);
+    L.sig = o;    o = align_up(o + (lut ? static_cast<size_t>(L.m_pad) * 4 : 0), kAlign);
     L.total = o;
     return L;
   }

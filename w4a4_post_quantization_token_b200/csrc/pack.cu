@@ -191,9 +191,14 @@ cudaError_t pack_act(const ActLayout& AL, int rank, const uint8_t* codes, const 
   const int K = static_cast<int>(AL.K);
   cudaError_t e;
   if ((e = cudaMemsetAsync(act, 0, AL.total, st)) != cudaSuccess) return e;
-  if ((e = cudaMemcpyAsync(act + AL.codes, codes, static_cast<size_t>(M) * (K / 2),
+  if ((e = cudaMemcpyAsync(act + AL.codes, codes, static_cast<size_t>(M) * (AL.lut ? K * 2 : K / 2),
                            cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
-  KQ_LAUNCH(k_sf_to_tiled, M * (K / kBlock), scales, M, K, act + AL.sf, sf_katoms(K));
+  if (AL.lut) {                                           // per-token sigma
+    if ((e = cudaMemcpyAsync(act + AL.sig, scales, static_cast<size_t>(M) * 4,
+                             cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
+  } else {
+    KQ_LAUNCH(k_sf_to_tiled, M * (K / kBlock), scales, M, K, act + AL.sf, sf_katoms(K));
+  }
   if (mu && (e = cudaMemcpyAsync(act + AL.mu, mu, static_cast<size_t>(M) * 4,
                                  cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
   if (rank > 0 && U)
@@ -206,14 +211,47 @@ cudaError_t unpack_act(const ActLayout& AL, int rank, const uint8_t* act, uint8_
   const int64_t M = AL.M;
   const int K = static_cast<int>(AL.K);
   cudaError_t e;
-  if (codes && (e = cudaMemcpyAsync(codes, act + AL.codes, static_cast<size_t>(M) * (K / 2),
+  if (codes && (e = cudaMemcpyAsync(codes, act + AL.codes, static_cast<size_t>(M) * (AL.lut ? K * 2 : K / 2),
                                     cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
-  if (scales)
+  if (scales && AL.lut) {
+    if ((e = cudaMemcpyAsync(scales, act + AL.sig, static_cast<size_t>(M) * 4,
+                             cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
+  } else if (scales) {
     KQ_LAUNCH(k_sf_from_tiled, M * (K / kBlock), act + AL.sf, M, K, sf_katoms(K), scales);
+  }
   if (mu && (e = cudaMemcpyAsync(mu, act + AL.mu, static_cast<size_t>(M) * 4,
                                  cudaMemcpyDeviceToDevice, st)) != cudaSuccess) return e;
   if (rank > 0 && U)
     KQ_LAUNCH(k_unpad_cols_bf16, M * rank, reinterpret_cast<const uint16_t*>(act + AL.u), M, rank, U);
+  return cudaSuccess;
+}
+
+// MXFP4 residual (internal layout) -> fp16 [N, K]: E2M1 magnitude x 2^(byte - 127), formed
+// exactly in float64 and rounded to nearest even fp16. One thread per 32-element block.
+__global__ void k_decode_residual_f16(const uint8_t* __restrict__ rcodes, const uint8_t* __restrict__ rsf,
+                                      int64_t N, int K, int64_t katoms, uint16_t* __restrict__ out) {
+  const int nb = K / kBlock;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= N * nb) return;
+  const int64_t n = t / nb;
+  const int b = static_cast<int>(t % nb);
+  // E2M1 magnitudes of codes 0..7 (OCP MX: exponent bias 1, one mantissa bit)
+  constexpr double kMag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+  const double sc = ldexp(1.0, static_cast<int>(rsf[sf_offset(n, b, katoms)]) - 127);
+  const uint8_t* c = rcodes + n * (K / 2) + b * 16;
+  uint16_t* o = out + n * K + b * kBlock;
+  for (int j = 0; j < kBlock; ++j) {
+    const uint32_t code = (c[j / 2] >> (4 * (j & 1))) & 15u;
+    const double v = (code & 8u) ? -kMag[code & 7u] * sc : kMag[code & 7u] * sc;
+    const __half h = __double2half(v);
+    o[j] = *reinterpret_cast<const uint16_t*>(&h);
+  }
+}
+
+cudaError_t decode_residual_f16(const WeightsLayout& WL, uint8_t* w, cudaStream_t st) {
+  const int K = static_cast<int>(WL.K);
+  KQ_LAUNCH(k_decode_residual_f16, WL.N * (K / kBlock), w + WL.rcodes, w + WL.rsf, WL.N, K,
+            sf_katoms(K), reinterpret_cast<uint16_t*>(w + WL.rf16));
   return cudaSuccess;
 }
 

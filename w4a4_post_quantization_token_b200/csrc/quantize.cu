@@ -122,7 +122,8 @@ __device__ __forceinline__ void encode_scaled2(const uint64_t (&v2)[16], float f
 // Transform + encode of one 32-element block (row r of the ring slot, block b). Writes the
 // codes (or, in debug mode, the transformed values) and returns the scale byte.
 // CENTER: 0 off, 1 centring, 2 LayerNorm then centring of the normalised token.
-template <int KIND, int CENTER, bool DEBUG_XT>
+// LUT: Lloyd-Max codebook out (ln = sigma, 1/sigma) instead of MXFP4.
+template <int KIND, int CENTER, bool DEBUG_XT, bool LUT>
 __device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const uint64_t (&Ap)[16],
                                                    const uint64_t (&Bp)[32], const uint8_t* rowb,
                                                    const uint8_t* tables, const uint8_t* lntab,
@@ -207,6 +208,40 @@ __device__ __forceinline__ uint32_t quantize_block(const QuantParams& p, const u
       o[q] = make_float4(f2lo(v2[2 * q]), f2hi(v2[2 * q]), f2lo(v2[2 * q + 1]), f2hi(v2[2 * q + 1]));
     return 0u;
   }
+  if (LUT) {
+    // |Xt| / sigma against the thresholds (a magnitude on a threshold takes the larger
+    // level), the level times sigma rounded to fp16, the sign of Xt (RPBH: of y times the
+    // channel sign) set on the result
+    const float cinv = KIND == 2 ? rs * ln.y : ln.y;
+    float mg[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) mg[i] = ln.x * p.lut_mag[i];
+    uint32_t out[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      float a, c2;
+      f2unpack(v2[q], a, c2);
+      uint32_t s0 = __float_as_uint(a) >> 31, s1 = __float_as_uint(c2) >> 31;
+      if (KIND == 2) {
+        const uint32_t mw = signs[4 * b + q / 4];
+        s0 ^= (mw >> (4 * (2 * (q % 4)) + 3)) & 1u;
+        s1 ^= (mw >> (4 * (2 * (q % 4) + 1) + 3)) & 1u;
+      }
+      const float ta = fabsf(a) * cinv, tb = fabsf(c2) * cinv;
+      float va = mg[0], vb = mg[0];
+#pragma unroll
+      for (int j = 0; j < 7; ++j) {
+        va = ta >= p.lut_thr[j] ? mg[j + 1] : va;
+        vb = tb >= p.lut_thr[j] ? mg[j + 1] : vb;
+      }
+      const __half2 h = __floats2half2_rn(va, vb);
+      out[q] = *reinterpret_cast<const uint32_t*>(&h) | (s0 << 15) | (s1 << 31);
+    }
+    uint4* o = reinterpret_cast<uint4*>(p.a16 + static_cast<size_t>(row) * p.K + b * kBlock);
+#pragma unroll
+    for (int v = 0; v < 4; ++v) o[v] = make_uint4(out[4 * v], out[4 * v + 1], out[4 * v + 2], out[4 * v + 3]);
+    return 0u;
+  }
   uint32_t c[4];
   uint32_t sbyte;
   if (KIND == 2) {
@@ -265,7 +300,7 @@ __device__ __forceinline__ void store_scales(const QuantParams& p, bool valid, i
 // once per CTA, as one bulk copy of a table prepared with the weights; the Kronecker
 // factors live in registers. Centring: the warp forms each row's mean (fp32 block sums,
 // fp64 across blocks), then all u * K/32 blocks of the unit are spread over the lanes.
-template <int KIND, int CENTER, bool DEBUG_XT>
+template <int KIND, int CENTER, bool DEBUG_XT, bool LUT>
 __global__ void __launch_bounds__(KIND == 1 ? 32 * kQMaxWarpsKron : 32 * kQMaxWarps, 1)
 k_quantize_rows(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -353,11 +388,11 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
     const uint8_t* ub = wbufs + static_cast<size_t>(s) * slot_bytes;
     const int64_t row0 = (l * G + blockIdx.x) * u;
     const int rows = static_cast<int>(min(static_cast<int64_t>(u), p.M - row0));
-    if (CENTER) {
+    if (CENTER || LUT) {
       for (int r = 0; r < rows; ++r) {
         const uint8_t* rowb = ub + static_cast<size_t>(r) * rstride;
         double part = 0.0;
-        for (int b = lane; b < nb; b += 32) {
+        for (int b = lane; CENTER && b < nb; b += 32) {
           uint64_t acc = 0;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -368,7 +403,7 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
           }
           part += static_cast<double>(f2lo(acc) + f2hi(acc));
         }
-        const double mu64 = warp_sum_f64(part) / static_cast<double>(p.K);
+        const double mu64 = CENTER ? warp_sum_f64(part) / static_cast<double>(p.K) : 0.0;
         const float mu_hi = static_cast<float>(mu64);
         const float mu_lo = static_cast<float>(mu64 - static_cast<double>(mu_hi));
         if (CENTER == 2) {
@@ -415,9 +450,38 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
               p.lnr[row0 + r] = static_cast<float>(rstd);
             }
           }
-        } else if (lane == 0) {
-          wmu[r] = make_float2(mu_hi, mu_lo);
-          p.mu[row0 + r] = mu_hi;
+        } else {
+          if (LUT) {
+            // sigma = RMS of the (centred) token, which the orthonormal rotation keeps:
+            // sum d^2 with d = (x - m_hi) - m_lo, fp32 per block, fp64 across blocks
+            const uint64_t mh = f2pack(mu_hi, mu_hi), ml = f2pack(mu_lo, mu_lo);
+            double pv = 0.0;
+            for (int b = lane; b < nb; b += 32) {
+              uint64_t av = 0;
+#pragma unroll
+              for (int c = 0; c < 4; ++c) {
+                const uint4 q = *reinterpret_cast<const uint4*>(rowb + swz64(static_cast<uint32_t>(b) * 64u + 16u * c));
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                  const uint64_t d = CENTER ? fsub2(fsub2(bf16x2_to_f2(w4[t]), mh), ml) : bf16x2_to_f2(w4[t]);
+                  av = ffma2(d, d, av);
+                }
+              }
+              pv += static_cast<double>(f2lo(av)) + static_cast<double>(f2hi(av));
+            }
+            const double sg = sqrt(warp_sum_f64(pv) / static_cast<double>(p.K));
+            const float sg32 = static_cast<float>(sg);
+            const float inv32 = sg > 0.0 ? static_cast<float>(1.0 / sg) : 0.f;
+            if (lane == 0) {
+              wln[r] = make_float4(sg32, inv32, 0.f, 0.f);
+              p.sig[row0 + r] = sg32;
+            }
+          }
+          if (lane == 0) {
+            wmu[r] = make_float2(mu_hi, mu_lo);
+            p.mu[row0 + r] = mu_hi;
+          }
         }
       }
       __syncwarp();
@@ -436,12 +500,12 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
         float mh = 0.f, ml = 0.f;
         float4 lr = make_float4(0.f, 0.f, 0.f, 0.f);
         if (CENTER) { const float2 m = wmu[r]; mh = m.x; ml = m.y; }
-        if (CENTER == 2) lr = wln[r];
-        sb = quantize_block<KIND, CENTER, DEBUG_XT>(p, Ap, Bp, ub + static_cast<size_t>(r) * rstride,
+        if (CENTER == 2 || LUT) lr = wln[r];
+        sb = quantize_block<KIND, CENTER, DEBUG_XT, LUT>(p, Ap, Bp, ub + static_cast<size_t>(r) * rstride,
                                                     tables, lntab, static_cast<int>(row0 + r), b, mh,
                                                     ml, lr);
       }
-      if (!DEBUG_XT) store_scales(p, valid, static_cast<int>(row0 + r), b, nb, nb_pad, sb);
+      if (!DEBUG_XT && !LUT) store_scales(p, valid, static_cast<int>(row0 + r), b, nb, nb_pad, sb);
       b += 32;
       while (b >= nb) { b -= nb; ++r; }
     }
@@ -459,10 +523,11 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
     const int nthr = NW * 32;
     for (int i = blockIdx.x * nthr + tid; i < pad_rows * wpr; i += G * nthr) {
       const int rr = p.M + i / wpr, w = i % wpr;
-      *reinterpret_cast<uint32_t*>(p.sf + sf_offset(rr, 4 * w, p.katoms)) = 0u;
+      if (!LUT) *reinterpret_cast<uint32_t*>(p.sf + sf_offset(rr, 4 * w, p.katoms)) = 0u;
       if (w == 0) {
         p.mu[rr] = 0.f;
         if (CENTER == 2) { p.lnm[rr] = 0.f; p.lnr[rr] = 0.f; }
+        if (LUT) p.sig[rr] = 0.f;
       }
     }
   }
@@ -701,10 +766,10 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
 // ----------------------------------------------------------------------------------
 // host launchers
 // ----------------------------------------------------------------------------------
-template <int KIND, int CENTER, bool DBG>
+template <int KIND, int CENTER, bool DBG, bool LUT = false>
 static cudaError_t launch_rows_t(const QuantParams& p, int num_sms, int block, size_t smem,
                                  cudaStream_t st) {
-  auto fn = k_quantize_rows<KIND, CENTER, DBG>;
+  auto fn = k_quantize_rows<KIND, CENTER, DBG, LUT>;
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -721,6 +786,14 @@ cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sm
   const int block = 32 * p.consumer_warps;
   const size_t smem = p.smem_bytes;
   const int kind = p.kind, c = p.center ? (p.ln ? 2 : 1) : 0;
+  // Lloyd-Max output (the debug entry stops before the encoder and takes the MXFP4 path)
+  if (p.lut && !debug_xt) {
+    if (kind == 0 && c == 0) return launch_rows_t<0, 0, false, true>(p, num_sms, block, smem, st);
+    if (kind == 0 && c == 1) return launch_rows_t<0, 1, false, true>(p, num_sms, block, smem, st);
+    if (kind == 2 && c == 0) return launch_rows_t<2, 0, false, true>(p, num_sms, block, smem, st);
+    if (kind == 2 && c == 1) return launch_rows_t<2, 1, false, true>(p, num_sms, block, smem, st);
+    return cudaErrorInvalidValue;
+  }
 #define KQ_DISPATCH(KD, C)                                                             \
   if (kind == KD && c == C)                                                            \
     return debug_xt ? launch_rows_t<KD, C, true>(p, num_sms, block, smem, st)          \
