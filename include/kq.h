@@ -207,8 +207,14 @@ kq_status kq_linear(const kq_layer_desc *desc, const void *weights, const void *
                     kq_stream_t stream);
 
 /* The same layer from HOST buffers: copies X (pinned host, bf16 [M, K]) to the device
- * buffer X_dev, runs kq_linear, and copies Y back into Y_host (pinned host). All three
- * steps are enqueued on `stream`; the call returns without waiting. */
+ * buffer X_dev [M, K], runs the layer, and copies Y back into Y_host (pinned host) from
+ * Y_dev [M, N]. For M >= 1024 the rows go in up to 8 chunks (a multiple of 128 rows,
+ * >= 512 each): the copy-in of a chunk, the kernels of the previous one and the copy-out
+ * of the one before run at the same time, the copies on two streams the library keeps
+ * per device (created on first use), ordered against `stream` with events. All work is
+ * ordered after the work already on `stream`, and work enqueued on `stream` after this
+ * call runs after all of it; the call returns without waiting. The device error word
+ * (kq_last_device_error) covers every chunk. */
 kq_status kq_linear_host(const kq_layer_desc *desc, const void *weights, const void *X_host,
                          void *X_dev, int32_t M, void *Y_host, void *Y_dev, int32_t out_dtype,
                          void *act, size_t act_bytes, kq_stream_t stream);

@@ -138,3 +138,32 @@ def test_linear_host_buffers(cuda_device):
     torch.cuda.synchronize()
     Yref = olayer.linear(inp["X"], inp["T"], w.center, prep)
     assert rel_fro(Yh.double().numpy(), Yref) <= 1e-3
+
+
+def test_linear_host_buffers_chunked(cuda_device):
+    """M >= 1024 goes through the chunked host pipeline (5 chunks of 640 rows, the last one
+    ragged): the device-buffer call's result up to the low-rank split, and the oracle's."""
+    import torch
+    import w4a4_post_quantization_token_b200 as kq
+    w, inp, prep = cached(2, M=2600, N=512)
+    L = make_layer(w, inp["T"])
+    wbuf = pack_oracle_weights(L, prep)
+    Xh = inp["X"].pin_memory()
+    Yh = torch.full((w.M, w.N), float("nan"), dtype=torch.float32).pin_memory()
+    Xd = torch.empty_like(Xh, device="cuda")
+    Yd = torch.empty((w.M, w.N), dtype=torch.float32, device="cuda")
+    act = torch.empty(kq.act_bytes(L, w.M), dtype=torch.uint8, device="cuda")
+    for _ in range(2):                               # the second call reuses the pipeline
+        kq.linear_host(L, wbuf, Xh, Xd, Yh, Yd, act)
+    torch.cuda.synchronize()
+    assert kq.last_device_error(L, act, w.M) == 0
+    Ydev = torch.empty((w.M, w.N), dtype=torch.float32, device="cuda")
+    kq.linear(L, wbuf, inp["X"].cuda(), Ydev, act)
+    torch.cuda.synchronize()
+    got = Yh.double().numpy()
+    assert np.all(np.isfinite(got))
+    # per-row arithmetic is the same, except that the low-rank kernel splits K by the
+    # number of rows it gets, so U's fp32 partial sums (and an occasional fp16 rounding of
+    # U) differ between a 640-row chunk and the 2600-row call
+    assert rel_fro(got, Ydev.cpu().double().numpy()) <= 2e-5
+    assert rel_fro(got, olayer.linear(inp["X"], inp["T"], w.center, prep)) <= 1e-3

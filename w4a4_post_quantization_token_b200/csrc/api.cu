@@ -17,7 +17,7 @@ using namespace kq;
 namespace {
 
 // ------------------------------------------------------------------ device checks --
-struct DeviceInfo { bool ok = false; int sms = 0; };
+struct DeviceInfo { bool ok = false; int sms = 0; int device = 0; };
 
 kq_status current_device(DeviceInfo* out) {
   int dev = 0;
@@ -35,6 +35,7 @@ kq_status current_device(DeviceInfo* out) {
     if (major != 10 || minor != 0) return KQ_ERR_NO_SM100;
     cache[dev].ok = true;
     cache[dev].sms = sms;
+    cache[dev].device = dev;
   }
   *out = cache[dev];
   return KQ_OK;
@@ -411,12 +412,13 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
 }
 
 kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* X, int M,
-                       uint8_t* act, cudaStream_t st, const DeviceInfo& di) {
+                       uint8_t* act, cudaStream_t st, const DeviceInfo& di, bool keep_err = false) {
   const WeightsLayout WL = wlayout(d);
   const ActLayout AL = alayout(d, M);
   QuantParams qp;
   kq_status s = fill_quant_params(d, weights, X, M, act, &qp, di);
   if (s != KQ_OK) return s;
+  qp.keep_err = keep_err ? 1 : 0;
   if (launch_quantize_rows(qp, false, di.sms, st) != cudaSuccess) return KQ_ERR_CUDA;
   if (d->rank > 0) {
     LowRankParams lp;
@@ -566,6 +568,50 @@ kq_status prepare_weights_impl(const kq_layer_desc* desc, const void* W_bf16, vo
   return write_ln_weights(desc, static_cast<uint8_t*>(weights), a.stream);
 }
 
+// Streams and events of the host-buffer entry, one set per device, created on first use.
+// The copies of one call run on two streams of their own (host-to-device, device-to-
+// host) so that they overlap each other and the kernels; kq_linear_host orders them
+// against the caller's stream with events.
+constexpr int kHostChunksMax = 8;
+struct HostPipe {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, done = nullptr;
+  cudaEvent_t ev_in[kHostChunksMax] = {}, ev_c[kHostChunksMax] = {};
+  std::mutex mu;
+  bool ok = false;
+};
+HostPipe* host_pipe(int device) {
+  static std::mutex m;
+  static HostPipe* pipes[64] = {};
+  if (device < 0 || device >= 64) return nullptr;
+  std::lock_guard<std::mutex> g(m);
+  if (!pipes[device]) {
+    HostPipe* h = new HostPipe;
+    bool ok = cudaStreamCreateWithFlags(&h->in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&h->out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&h->done, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < kHostChunksMax; ++i)
+      ok = cudaEventCreateWithFlags(&h->ev_in[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h->ev_c[i], cudaEventDisableTiming) == cudaSuccess;
+    h->ok = ok;
+    pipes[device] = h;
+  }
+  return pipes[device]->ok ? pipes[device] : nullptr;
+}
+
+// kq_linear's device work with the device error word kept (row chunks after the first)
+kq_status linear_dev(const kq_layer_desc* desc, const void* weights, const void* X, int32_t M,
+                     void* Y, int32_t out_dtype, void* act, size_t act_bytes, cudaStream_t st,
+                     const DeviceInfo& di, bool keep_err) {
+  if (M <= 0 || !weights || !X || !act || !Y) return KQ_ERR_INVALID_ARG;
+  if (!aligned(weights) || !aligned(X) || !aligned(act) || !aligned(Y)) return KQ_ERR_ALIGNMENT;
+  if (act_bytes < alayout(desc, M).total) return KQ_ERR_WORKSPACE_TOO_SMALL;
+  kq_status s = run_quantize(desc, weights, X, M, static_cast<uint8_t*>(act), st, di, keep_err);
+  if (s != KQ_OK) return s;
+  return run_gemm(desc, weights, static_cast<const uint8_t*>(act), M, Y, out_dtype, st, di);
+}
+
 }  // namespace
 
 extern "C" {
@@ -692,14 +738,52 @@ kq_status kq_linear_host(const kq_layer_desc* desc, const void* weights, const v
   kq_status s = check_desc(desc);
   if (s != KQ_OK) return s;
   if (!X_host || !Y_host || !X_dev || !Y_dev || M <= 0) return KQ_ERR_INVALID_ARG;
+  if (out_dtype != KQ_OUT_F32 && out_dtype != KQ_OUT_BF16) return KQ_ERR_INVALID_ARG;
+  if (!weights || !act) return KQ_ERR_INVALID_ARG;
+  if (!aligned(weights) || !aligned(X_dev) || !aligned(Y_dev) || !aligned(act)) return KQ_ERR_ALIGNMENT;
+  if (act_bytes < alayout(desc, M).total) return KQ_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t xb = static_cast<size_t>(M) * desc->K * 2;
-  const size_t yb = static_cast<size_t>(M) * desc->N * (out_dtype == KQ_OUT_BF16 ? 2 : 4);
-  if (cudaMemcpyAsync(X_dev, X_host, xb, cudaMemcpyHostToDevice, st) != cudaSuccess)
+  const size_t xrow = static_cast<size_t>(desc->K) * 2;
+  const size_t yrow = static_cast<size_t>(desc->N) * (out_dtype == KQ_OUT_BF16 ? 2 : 4);
+  // Rows in chunks of a 128 multiple (>= 512 rows, <= 8 chunks): the copy-in of chunk
+  // i + 1, the kernels of chunk i and the copy-out of chunk i - 1 run at the same time
+  // (PCIe moves both directions at once). One chunk: everything on `stream`.
+  int nch = M >= 1024 ? std::min(kHostChunksMax, M / 512) : 1;
+  const int C = static_cast<int>(align_up(static_cast<size_t>(cdiv(M, nch)), 128));
+  nch = static_cast<int>(cdiv(M, C));
+  HostPipe* hp = nch > 1 ? host_pipe(di.device) : nullptr;
+  if (!hp) {
+    if (cudaMemcpyAsync(X_dev, X_host, M * xrow, cudaMemcpyHostToDevice, st) != cudaSuccess)
+      return KQ_ERR_CUDA;
+    if ((s = linear_dev(desc, weights, X_dev, M, Y_dev, out_dtype, act, act_bytes, st, di, false)) != KQ_OK)
+      return s;
+    if (cudaMemcpyAsync(Y_host, Y_dev, M * yrow, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+      return KQ_ERR_CUDA;
+    return KQ_OK;
+  }
+  std::lock_guard<std::mutex> g(hp->mu);
+  if (cudaEventRecord(hp->start, st) != cudaSuccess || cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
     return KQ_ERR_CUDA;
-  s = kq_linear(desc, weights, X_dev, M, Y_dev, out_dtype, act, act_bytes, stream);
-  if (s != KQ_OK) return s;
-  if (cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+  for (int i = 0; i < nch; ++i) {
+    const size_t r0 = static_cast<size_t>(i) * C;
+    const int rows = static_cast<int>(std::min<size_t>(C, M - r0));
+    if (cudaMemcpyAsync(static_cast<uint8_t*>(X_dev) + r0 * xrow, static_cast<const uint8_t*>(X_host) + r0 * xrow,
+                        rows * xrow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+        cudaEventRecord(hp->ev_in[i], hp->in) != cudaSuccess || cudaStreamWaitEvent(st, hp->ev_in[i], 0) != cudaSuccess)
+      return KQ_ERR_CUDA;
+    if ((s = linear_dev(desc, weights, static_cast<uint8_t*>(X_dev) + r0 * xrow, rows,
+                        static_cast<uint8_t*>(Y_dev) + r0 * yrow, out_dtype, act, act_bytes, st, di,
+                        i > 0)) != KQ_OK)
+      return s;
+    if (cudaEventRecord(hp->ev_c[i], st) != cudaSuccess || cudaStreamWaitEvent(hp->out, hp->ev_c[i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(static_cast<uint8_t*>(Y_host) + r0 * yrow, static_cast<const uint8_t*>(Y_dev) + r0 * yrow,
+                        rows * yrow, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
+      return KQ_ERR_CUDA;
+  }
+  if (cudaEventRecord(hp->done, hp->out) != cudaSuccess || cudaStreamWaitEvent(st, hp->done, 0) != cudaSuccess)
     return KQ_ERR_CUDA;
   return KQ_OK;
 }

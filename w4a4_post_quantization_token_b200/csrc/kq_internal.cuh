@@ -51,6 +51,8 @@ struct QuantParams {
   uint32_t lntab_off;          // its shared-memory offset (128-byte aligned)
   float* lnm;                  // out: per-token mean of x [m_pad]
   float* lnr;                  // out: per-token 1/sqrt(v + eps) [m_pad]
+  int keep_err;                // 1: leave the device error word as it is (later row chunks
+                               //    of one call), 0: clear it first
   int lut;                     // Lloyd-Max activations: fp16 operand out, no block scales
   float lut_mag[8];            //   positive codebook levels (ascending)
   float lut_thr[7];            //   thresholds between them

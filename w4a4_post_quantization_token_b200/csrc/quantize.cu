@@ -327,7 +327,7 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
   // stream order (after every kernel of the previous call has finished), and a kernel of
   // this call can set the word only when one of its waits has run 2 s, long after CTA 0
   // has started, so clearing it here cannot lose an error.
-  if (blockIdx.x == 0 && tid == 0 && p.err != nullptr) *p.err = 0u;
+  if (blockIdx.x == 0 && tid == 0 && p.err != nullptr && !p.keep_err) *p.err = 0u;
 
   uint64_t Ap[16], Bp[32];
   if (KIND == 1) {
