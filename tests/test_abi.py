@@ -177,3 +177,12 @@ def test_library_codebook_matches_the_oracle():
     pos, pth = lm.magnitudes()
     np.testing.assert_allclose(lv, pos, rtol=1e-13, atol=0)
     np.testing.assert_allclose(th, pth, rtol=1e-13, atol=0)
+
+
+def test_rpbh_largest_k():
+    """The RPBH gather table holds 16-bit byte offsets into a staged row: K <= 32736."""
+    ok = kq.Layer(32736, 64, 0, False, _rpbh(32736))
+    assert kq.weights_bytes(ok) > 0
+    big = kq.Layer(32768, 64, 0, False, _rpbh(32768))
+    assert kq.weights_bytes(big) == 0
+    assert kq.lib.kq_quantize_act(big.desc, None, None, 4, None, 0, None) == 2

@@ -74,6 +74,8 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 // ---------------------------------------------------------------- validation --------
 bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
 
+constexpr int kRpbhMaxK = 32736;    // largest K % 32 == 0 with 2 K < 65536
+
 kq_status check_desc(const kq_layer_desc* d) {
   if (!d) return KQ_ERR_INVALID_ARG;
   if (d->K <= 0 || d->N <= 0 || d->rank < 0) return KQ_ERR_INVALID_ARG;
@@ -89,11 +91,13 @@ kq_status check_desc(const kq_layer_desc* d) {
       break;
     case KQ_T_RPBH: {
       if (!d->t.perm || !d->t.sign) return KQ_ERR_INVALID_ARG;
-      std::vector<char> seen(static_cast<size_t>(d->K), 0);
+      // the gather table holds 16-bit byte offsets into a staged row: 2 K < 65536
+      if (d->K > kRpbhMaxK) return KQ_ERR_UNSUPPORTED_SHAPE;
+      uint64_t seen[kRpbhMaxK / 64 + 1] = {};            // on the stack: no allocation per call
       for (int k = 0; k < d->K; ++k) {
         const int32_t p = d->t.perm[k];
-        if (p < 0 || p >= d->K || seen[p]) return KQ_ERR_INVALID_ARG;
-        seen[p] = 1;
+        if (p < 0 || p >= d->K || ((seen[p >> 6] >> (p & 63)) & 1u)) return KQ_ERR_INVALID_ARG;
+        seen[p >> 6] |= 1ull << (p & 63);
         if (d->t.sign[k] != 1 && d->t.sign[k] != -1) return KQ_ERR_INVALID_ARG;
       }
       break;
@@ -336,7 +340,6 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   // each row is staged in a 512-byte aligned slot row (its own 64-byte swizzle pattern),
   // loaded in boxes of up to 256 lines
   const uint32_t rstride = static_cast<uint32_t>(align_up(static_cast<size_t>(K) * 2, 512));
-  if (d->t.kind == KQ_T_RPBH && K * 2 > 65535) return KQ_ERR_UNSUPPORTED_SHAPE;
   int box = 1;
   for (int c = 1; c <= 256 && c <= nb; ++c) if (nb % c == 0) box = c;
   p->box_lines = box;
@@ -767,25 +770,29 @@ kq_status kq_linear_host(const kq_layer_desc* desc, const void* weights, const v
   if (cudaEventRecord(hp->start, st) != cudaSuccess || cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
       cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
     return KQ_ERR_CUDA;
-  for (int i = 0; i < nch; ++i) {
+  for (int i = 0; i < nch && s == KQ_OK; ++i) {
     const size_t r0 = static_cast<size_t>(i) * C;
     const int rows = static_cast<int>(std::min<size_t>(C, M - r0));
     if (cudaMemcpyAsync(static_cast<uint8_t*>(X_dev) + r0 * xrow, static_cast<const uint8_t*>(X_host) + r0 * xrow,
                         rows * xrow, cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
-        cudaEventRecord(hp->ev_in[i], hp->in) != cudaSuccess || cudaStreamWaitEvent(st, hp->ev_in[i], 0) != cudaSuccess)
-      return KQ_ERR_CUDA;
+        cudaEventRecord(hp->ev_in[i], hp->in) != cudaSuccess || cudaStreamWaitEvent(st, hp->ev_in[i], 0) != cudaSuccess) {
+      s = KQ_ERR_CUDA;
+      break;
+    }
     if ((s = linear_dev(desc, weights, static_cast<uint8_t*>(X_dev) + r0 * xrow, rows,
                         static_cast<uint8_t*>(Y_dev) + r0 * yrow, out_dtype, act, act_bytes, st, di,
                         i > 0)) != KQ_OK)
-      return s;
+      break;
     if (cudaEventRecord(hp->ev_c[i], st) != cudaSuccess || cudaStreamWaitEvent(hp->out, hp->ev_c[i], 0) != cudaSuccess ||
         cudaMemcpyAsync(static_cast<uint8_t*>(Y_host) + r0 * yrow, static_cast<const uint8_t*>(Y_dev) + r0 * yrow,
                         rows * yrow, cudaMemcpyDeviceToHost, hp->out) != cudaSuccess)
-      return KQ_ERR_CUDA;
+      s = KQ_ERR_CUDA;
   }
-  if (cudaEventRecord(hp->done, hp->out) != cudaSuccess || cudaStreamWaitEvent(st, hp->done, 0) != cudaSuccess)
+  // whatever was enqueued, the caller's stream is ordered after both copy streams
+  if (cudaEventRecord(hp->ev_c[0], hp->in) != cudaSuccess || cudaStreamWaitEvent(st, hp->ev_c[0], 0) != cudaSuccess ||
+      cudaEventRecord(hp->done, hp->out) != cudaSuccess || cudaStreamWaitEvent(st, hp->done, 0) != cudaSuccess)
     return KQ_ERR_CUDA;
-  return KQ_OK;
+  return s;
 }
 
 kq_status kq_weights_pack(const kq_layer_desc* desc, const void* r_codes, const void* r_scales,
