@@ -165,3 +165,20 @@ def test_prepare_on_gpu(cuda_device):
     # the GPU's own SVD and residual encode differ from the oracle's at rounding level
     # (their parity is tested with the MXFP4 layer); that adds to the bound here
     _check_layer(w, inp, prep, *_linear(L, wbuf, inp["X"], w.N), tol=2e-3)
+
+
+@pytest.mark.parametrize("index", [2, 4])
+def test_layer_full_size_sampled(cuda_device, index):
+    """The full RPBH workloads in the bench's launch configuration; the oracle checks 48
+    sampled rows (incl. the last ones) on the GPU's validated decisions."""
+    import w4a4_post_quantization_token_b200 as kq
+    from tests.kqtest import cached
+    w, inp, prep = cached(index)
+    L = kq.Layer(w.K, w.N, w.rank, w.center, inp["T"], codebook="lloydmax")
+    wbuf = pack_oracle_weights(L, prep)
+    Y, A, sig = _linear(L, wbuf, inp["X"], w.N)
+    rng = np.random.default_rng(index)
+    rows = np.unique(np.concatenate([rng.choice(w.M, 40, replace=False),
+                                     np.arange(max(0, w.M - 8), w.M)]))
+    sub = {"X": inp["X"][rows], "T": inp["T"]}
+    _check_layer(workload(index, M=len(rows)), sub, prep, Y[rows], A[rows], sig[rows])

@@ -153,3 +153,21 @@ def test_front_end_is_not_the_plain_layer(cuda_device):
     Lp = kq.Layer(w.K, w.N, w.rank, True, inp["T"])
     plain = _run_linear(Lp, pack_oracle_weights(Lp, prep), inp["X"].cuda(), w.N)
     assert rel_fro(Yg, plain) > 0.1
+
+
+@pytest.mark.parametrize("index", [2, 3, 5])
+def test_layer_full_size_sampled(cuda_device, index):
+    """Full workloads (centring on) with the front-end, in the bench's launch
+    configuration; the oracle checks 48 sampled rows (incl. the last ones)."""
+    import w4a4_post_quantization_token_b200 as kq
+    from tests.kqtest import cached
+    w, inp, prep = cached(index)
+    ln = make_layernorm(w)
+    L = kq.Layer(w.K, w.N, w.rank, True, inp["T"], layernorm=ln)
+    wbuf = pack_oracle_weights(L, prep)
+    Yg = _run_linear(L, wbuf, inp["X"].cuda(), w.N)
+    rng = np.random.default_rng(index)
+    rows = np.unique(np.concatenate([rng.choice(w.M, 40, replace=False),
+                                     np.arange(max(0, w.M - 8), w.M)]))
+    Y = oln.layernorm(inp["X"][rows].double().numpy(), ln["gamma"], ln["beta"], ln["eps"])
+    assert rel_fro(Yg[rows], olayer.linear(Y, inp["T"], True, prep)) <= 1e-3
