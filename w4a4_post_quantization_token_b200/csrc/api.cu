@@ -447,6 +447,9 @@ kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* 
     lp.mu = d->center ? reinterpret_cast<const float*>(act + AL.mu) : nullptr;
     lp.u = reinterpret_cast<uint16_t*>(act + AL.u);
     lp.M = M; lp.K = d->K; lp.split = u_split(M, d->K);
+    // a quantize CTA and a 3-stage low-rank CTA share an SM only when the quantize shape
+    // was chosen for it; otherwise the low-rank grid runs on SMs of its own: deep ring
+    lp.deep = qp.smem_bytes + kLowRankSmemBytes + 2 * kSmemPerBlockReserved > kSmemPerSM ? 1 : 0;
     lp.err = reinterpret_cast<uint32_t*>(act + AL.err);
     if (launch_lowrank_u(lp, st) != cudaSuccess) return KQ_ERR_CUDA;
   }

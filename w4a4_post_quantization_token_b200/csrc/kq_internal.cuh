@@ -68,6 +68,7 @@ struct LowRankParams {
   const float* c1;             // [64]
   const float* mu;             // [M] token means (null without centring)
   uint16_t* u;                 // U [M, 64] fp16
+  int deep;                    // 1: the quantize CTAs leave no room on the SM, use the deep ring
   int ln;                      // LayerNorm front-end: L1 map is diag(gamma) L1', and
   const float* cg;             //   U = rstd acc - rstd m cg + cb - mu c1 with cg = gamma^T L1'
   const float* cb;             //   and cb = beta^T L1' [64]

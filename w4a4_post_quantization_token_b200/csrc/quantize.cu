@@ -581,6 +581,9 @@ constexpr uint32_t kABytes = kTileM * 128;       // 16 KB
 constexpr uint32_t kBBytes = kUCols * 128;       // 16 KB
 constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kSmemBytes = 1024 + kStages * kStageBytes + 1024;
+// when the quantize kernel's shape leaves no room beside it, the ring is deeper
+constexpr int kStagesDeep = 6;
+constexpr uint32_t smem_bytes(int ns) { return 1024 + ns * kStageBytes + 1024; }
 constexpr uint32_t kTmemCols = 128;
 static_assert(kSmemBytes == kLowRankSmemBytes, "shared-memory footprint the quantize shape leaves room for");
 }  // namespace lowrank
@@ -638,8 +641,10 @@ __device__ __forceinline__ void lowrank_finish(const LowRankParams& p, const flo
   }
 }
 
+template <int NS>
 __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ LowRankParams p) {
   using namespace lowrank;
+  constexpr int kStages = NS;                          // TMA ring depth
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // no extra alignment offset: every CTA of a cluster must use the same smem offsets
   uint8_t* smem = smem_raw;
@@ -654,9 +659,9 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
   const int mt = blockIdx.x, ks = blockIdx.y, S = gridDim.y;
   const int m0 = mt * kTileM;
   const int KT = static_cast<int>(cdiv(p.K, kChunkK));
-  const int k_begin = static_cast<int>((static_cast<int64_t>(KT) * ks) / S);
-  const int k_end = static_cast<int>((static_cast<int64_t>(KT) * (ks + 1)) / S);
-  const int nk = k_end - k_begin;
+  // the S CTAs of a row tile take the 64-element K chunks in turn (chunk i S + ks), so
+  // that at any time they read neighbouring 128-byte pieces of the same rows
+  const int nk = KT > ks ? (KT - ks + S - 1) / S : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
@@ -681,8 +686,9 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
           break;
         uint8_t* a = stage0 + s * kStageBytes;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
-        tma_load_2d(a, &p.tmap_x, (k_begin + i) * kChunkK, m0, &full[s]);
-        tma_load_2d(a + kABytes, &p.tmap_l1, (k_begin + i) * kChunkK, 0, &full[s]);
+        const int kc = i * S + ks;
+        tma_load_2d(a, &p.tmap_x, kc * kChunkK, m0, &full[s]);
+        tma_load_2d(a + kABytes, &p.tmap_l1, kc * kChunkK, 0, &full[s]);
       }
     }
   } else if (warp == 1) {
@@ -816,13 +822,15 @@ cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint
 
 cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st) {
   using namespace lowrank;
-  cudaError_t e = cudaFuncSetAttribute(k_lowrank_u, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(kSmemBytes));
+  auto fn = p.deep ? k_lowrank_u<kStagesDeep> : k_lowrank_u<kStages>;
+  const uint32_t smem = smem_bytes(p.deep ? kStagesDeep : kStages);
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(cdiv(p.M, kTileM)), static_cast<unsigned>(p.split));
   cfg.blockDim = dim3(192);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -833,7 +841,7 @@ cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  e = cudaLaunchKernelEx(&cfg, k_lowrank_u, p);
+  e = cudaLaunchKernelEx(&cfg, fn, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
