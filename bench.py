@@ -230,6 +230,34 @@ def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = No
     return done / dt, done, dt
 
 
+def oracle_stage_seconds(w, inp, prep, rows: int = 256) -> dict:
+    """Wall time of the oracle's steps on the first `rows` tokens, per 1000 tokens: centring
+    and block transform, MXFP4 encode (with the float32 rounding of its input), the low-rank
+    input U, and the fp64 contraction (decode and the three terms)."""
+    from oracle import bf16 as obf16
+    from oracle import layer as olayer
+    from oracle import mxfp4 as omx
+    from oracle import transforms as otr
+    X = inp["X"][:rows].double().numpy()
+    out = {}
+    t0 = time.perf_counter()
+    mu, Xc = olayer.center(X, w.center)
+    Xt = otr.apply(Xc, inp["T"])
+    t1 = time.perf_counter()
+    codes, scales = omx.encode(obf16.round_f32(Xt))
+    t2 = time.perf_counter()
+    U = Xt @ prep["L1"]
+    t3 = time.perf_counter()
+    olayer.linear_from_parts({"codes": codes, "scales": scales, "U": U, "mu": mu}, prep)
+    t4 = time.perf_counter()
+    k = 1000.0 / rows
+    out["transform"] = (t1 - t0) * k
+    out["encode"] = (t2 - t1) * k
+    out["lowrank_input"] = (t3 - t2) * k
+    out["contraction"] = (t4 - t3) * k
+    return out
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -509,6 +537,8 @@ def main():
         cpu = {"value": v, "unit": "tokens/s", "cores": blas_threads(), "kind": "oracle",
                "sample": f"first {rows} of {w.M} tokens ({dt:.1f} s, fp64 NumPy, weights "
                          f"prepared beforehand)"}
+        if ln is None and not lut:
+            cpu["stage_seconds_per_1k_tokens"] = oracle_stage_seconds(w, inp, prep)
 
     comparator = None
     if not args.no_comparator:

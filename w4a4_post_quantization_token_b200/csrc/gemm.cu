@@ -27,6 +27,11 @@
 //              128-byte-swizzled staging tile in shared memory, TMA-store it (async).
 // A 192-wide tile whose first row sits in the middle of a 128-row scale atom reads its
 // B scales two TMEM columns further on. No TMA multicast is used anywhere.
+//
+// Codebook variant (template F16): the tensor cores have no format for a Lloyd-Max
+// codebook (OrbitQuant section 03), so those layers hand the contraction decoded fp16
+// operands (the activation as fp16(sigma level), the residual decoded offline) and the
+// main loop runs kind::f16 MMAs over 64-element k-tiles; everything else is shared.
 #include <cuda_bf16.h>
 
 #include "kq_internal.cuh"

@@ -11,7 +11,10 @@
 //    or gather + 32-point fast Walsh-Hadamard + sign (OrbitQuant commentary, section 03,
 //    RPBH(X) = X P H D), or a per-channel multiply by SmoothQuant inverse scales (the
 //    comparator of KroQuant section 02). MXFP4 encoding as in encode.cuh (KroQuant
-//    section 03).
+//    section 03), or (template LUT) the nearest level of a 16-level Lloyd-Max codebook
+//    of N(0, 1) for Xt / sigma with sigma the RMS of the centred token (OrbitQuant
+//    section 03; CentriQ abstract: the per-token scale in closed form), stored as the
+//    fp16 operand the contraction takes.
 //  * k_lowrank_u -- U = X L1' - mu c1 (SVDQuant explainer, section 3: the low-rank branch
 //    runs on the high-precision input) as a tcgen05 bf16 GEMM: TMA loads 128x64 tiles of
 //    X and of [L1'_hi; L1'_lo], the MMA accumulates 128 x 128 in TMEM, the epilogue forms
