@@ -114,7 +114,13 @@ typedef struct {
  * kq_prepare_weights / kq_weights_pack, which copy them into the prepared weights with
  * the low-rank map diag(gamma) L1' and the sums gamma^T L1', beta^T L1' (KQ_ERR_INVALID_ARG
  * there if a pointer is null or a value is not finite); later calls need on and eps only.
- * The activation workspace then also holds each token's m and 1/sqrt(v + eps). */
+ * The activation workspace then also holds each token's m and 1/sqrt(v + eps) (0 for a
+ * token with zero variance, which normalises to beta exactly).
+ * Conditioning: the low-rank input is formed from raw x as
+ * rstd (x diag(gamma) L1' - m gamma^T L1') + beta^T L1' - mean(y) c1, so its absolute error
+ * is about 2^-24 (|m| / sqrt(v + eps)) sum_k |gamma_k L1'_k| from fp32 accumulation: small
+ * for tokens whose mean is within a few standard deviations of zero (DiT residual streams),
+ * large for nearly constant tokens with a large mean. */
 typedef struct {
   int32_t on;            /* 1: front-end on */
   float eps;             /* > 0 */

@@ -360,9 +360,12 @@ __global__ void k_ln_fold(const uint16_t* __restrict__ l1t, const float* __restr
                      bf16_bits_to_f64(l1t[static_cast<size_t>(kRankPad + t) * K + k]);
     const double vg = static_cast<double>(gamma[k]) * v;
     const uint16_t hi = f64_to_bf16_bits(vg);
+    const uint16_t lo = f64_to_bf16_bits(vg - bf16_bits_to_f64(hi));
     l1gt[static_cast<size_t>(t) * K + k] = hi;
-    l1gt[static_cast<size_t>(kRankPad + t) * K + k] = f64_to_bf16_bits(vg - bf16_bits_to_f64(hi));
-    sg += vg;
+    l1gt[static_cast<size_t>(kRankPad + t) * K + k] = lo;
+    // gamma^T L1' from the stored pair, the values the MMA multiplies x by: m gamma^T L1'
+    // then cancels x diag(gamma) L1' up to fp32 accumulation only
+    sg += bf16_bits_to_f64(hi) + bf16_bits_to_f64(lo);
     sb += static_cast<double>(beta[k]) * v;
   }
   __shared__ double rg[256], rb[256];

@@ -449,8 +449,10 @@ k_quantize_rows(const __grid_constant__ QuantParams p) {
             wln[r] = make_float4(static_cast<float>(rstd), my_hi, my_lo, 0.f);
             p.mu[row0 + r] = my_hi;
             if (p.lnm != nullptr) {                  // null in the debug entry
+              // a token with zero variance normalises to beta exactly: its low-rank input
+              // is beta^T L1' - mean(y) c1, so the epilogue gets no rstd term for it
               p.lnm[row0 + r] = mu_hi;
-              p.lnr[row0 + r] = static_cast<float>(rstd);
+              p.lnr[row0 + r] = var > 0.0 ? static_cast<float>(rstd) : 0.f;
             }
           }
         } else {
