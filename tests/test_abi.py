@@ -186,3 +186,14 @@ def test_rpbh_largest_k():
     big = kq.Layer(32768, 64, 0, False, _rpbh(32768))
     assert kq.weights_bytes(big) == 0
     assert kq.lib.kq_quantize_act(big.desc, None, None, 4, None, 0, None) == 2
+
+
+def test_binding_fails_loudly_without_the_library():
+    """The product path has no fallback: without libkq.so next to it the package does not
+    import (executed here from its source with a location that holds no library)."""
+    import types
+    src_path = os.path.join(os.path.dirname(kq.__file__), "__init__.py")
+    mod = types.ModuleType("kq_without_library")
+    mod.__file__ = os.path.join(os.path.dirname(kq.__file__), "no_such_dir", "__init__.py")
+    with pytest.raises(ImportError, match="libkq.so not found"):
+        exec(compile(open(src_path).read(), mod.__file__, "exec"), mod.__dict__)
