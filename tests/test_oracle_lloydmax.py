@@ -2,6 +2,8 @@
 two-level closed form, the optimality conditions and the distortion by independent
 numerical quadrature, a brute-force nearest-level encoder, the scale invariance of the
 per-token sigma under the orthonormal rotation, and the fp16 operand rounding."""
+import os
+
 import numpy as np
 import pytest
 from scipy import integrate, stats
@@ -10,14 +12,23 @@ from oracle import lloydmax as lm
 from oracle import transforms
 from synthetic import make_inputs, workload
 
-# Max (1960), "Quantizing for minimum distortion", Table I, N = 16: the positive output
-# levels (the quantizer is symmetric), printed to 4 decimals.
-MAX_1960_N16 = [0.1284, 0.3881, 0.6568, 0.9424, 1.256, 1.618, 2.069, 2.733]
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "lloydmax_gaussian16.txt")
+
+
+def _max_table():
+    """Max (1960), Table I, N = 16 (tests/golden/lloydmax_gaussian16.txt): the positive
+    decision levels and output levels, 4 decimals."""
+    rows = [ln.split() for ln in open(GOLDEN) if ln.strip() and not ln.startswith("#")]
+    x = np.array([float(r[0]) for r in rows])
+    y = np.array([float(r[1]) for r in rows])
+    return x, y
 
 
 def test_matches_published_table():
     lv, th = lm.gaussian_lloyd_max(16)
-    np.testing.assert_allclose(lv[8:], MAX_1960_N16, atol=6e-4)
+    x, y = _max_table()
+    np.testing.assert_allclose(lv[8:], y, atol=6e-4)
+    np.testing.assert_allclose(th[7:], x, atol=6e-4)            # th[7] = 0: the sign decision
     np.testing.assert_array_equal(lv[:8], -lv[8:][::-1])                # symmetric
 
 
