@@ -1,9 +1,35 @@
 """Pins of the LayerNorm front-end oracle: a hand-computed row, the defining moments,
 invariance to a per-token shift, the affine, and the algebraic decomposition the GPU's
 low-rank kernel uses to form y L1' from raw activations."""
+import os
+
 import numpy as np
 
 from oracle import layernorm as ln
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "layernorm_rows.txt")
+
+
+def _golden():
+    cases, cur = [], None
+    for line in open(GOLDEN):
+        t = line.split()
+        if not t or t[0].startswith("#"):
+            continue
+        if t[0] == "case":
+            cur = {"name": t[1]}
+            cases.append(cur)
+        else:
+            cur[t[0]] = np.array([float(v) for v in t[1:]])
+    return cases
+
+
+def test_golden_rows():
+    cases = _golden()
+    assert len(cases) == 3
+    for c in cases:
+        y = ln.layernorm(c["x"][None, :], c["gamma"], c["beta"], float(c["eps"][0]))
+        np.testing.assert_allclose(y[0], c["y"], rtol=1e-15, atol=1e-15, err_msg=c["name"])
 
 
 def test_hand_row():
