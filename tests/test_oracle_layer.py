@@ -133,3 +133,46 @@ def test_centering_helps_with_token_shift():
     err_c = np.linalg.norm(layer.linear(X, inp["T"], True, prep) - Y) / np.linalg.norm(Y)
     err_n = np.linalg.norm(layer.linear(X, inp["T"], False, prep) - Y) / np.linalg.norm(Y)
     assert err_c < err_n
+
+
+@pytest.mark.parametrize("law,kind", [(1, "kron"), (2, "rpbh")])
+def test_exact_rank_weight_is_carried_by_the_lowrank_branch(law, kind):
+    """A weight of exact rank r, W = B1 B2, with rank r kept (SVDQuant section 3): the
+    transform-folded weight W' = P^{-1} W has rank r too, so the 16-bit factors hold all
+    of it and the 4-bit residual R = W' - L1 L2 holds only their bf16 rounding (about
+    2^-8 of W'). The layer output is then X W up to the MXFP4 error of the small product
+    Xt R: Y - X W = deq(Q(Xt)) deq(Q(R)) - Xt R, well under 1e-2 of X W. The pin is the
+    identity Xt L1 L2 + Xt R + mu s = X W (centring restores mu s exactly, the transform
+    cancels against its fold): dropping the U L2 term, forming U from the centred input
+    before the transform instead of Xt, or losing mu s each move Y by O(1) of X W, which
+    the test checks on the same data."""
+    M, K, N, r = 24, 64, 40, 4
+    rng = np.random.default_rng(11)
+    B1 = rng.integers(-3, 4, size=(K, r)).astype(np.float64) * 2.0 ** -3
+    B2 = rng.integers(-3, 4, size=(r, N)).astype(np.float64) * 2.0 ** -4
+    W = B1 @ B2
+    assert np.linalg.matrix_rank(W) == r
+    w = workload(law, M=M, K=K, N=N, rank=r, transform=kind, center=True)
+    inp = make_inputs(w)
+    X = inp["X"].double().numpy()
+    T = inp["T"]
+    prep = layer.prepare(W, T, r)
+    # the residual is only the rounding of the factors
+    assert np.linalg.norm(prep["R"]) < 2.0 ** -7 * np.linalg.norm(prep["Wp"])
+    act = layer.quantize_act(X, T, True, prep)
+    Y = layer.linear_from_parts(act, prep)
+    XW = X @ W
+    nrm = np.linalg.norm(XW)
+    err = np.linalg.norm(Y - XW) / nrm
+    assert err < 1e-2, err
+    # each plausible slip moves the output by O(1)
+    Xq = mxfp4.decode(act["codes"], act["scales"])
+    Rq = mxfp4.decode(prep["r_codes"], prep["r_scales"]).T
+    no_lowrank = Xq @ Rq + np.outer(act["mu"], prep["s"])
+    u_before_transform = Xq @ Rq + (act["Xc"] @ prep["L1"]) @ prep["L2"] + np.outer(act["mu"], prep["s"])
+    no_restore = Xq @ Rq + act["U"] @ prep["L2"]
+    for wrong in (no_lowrank, no_restore):
+        assert np.linalg.norm(wrong - XW) / nrm > 0.2
+    # the transform is close to the identity for the Kronecker law (I + N(0, 0.1)
+    # factors), so forming U before it is a smaller, still clearly visible slip
+    assert np.linalg.norm(u_before_transform - XW) / nrm > 10 * err
