@@ -7,11 +7,12 @@ centring, block transform, MXFP4 quantization and the low-rank input (quantize k
 then the block-scaled FP4 GEMM with the fused low-rank and rank-1 branches. The weights
 are prepared once, offline (reported separately as prepare_ms, not in tokens/s).
 
-Default workload: PixArt-Sigma-shaped MLP fc1 (M=4096 tokens, K=1152, N=4608, permuted
-block-Hadamard transform, rank-32 branch), bf16 output. Inputs are seeded synthetic
-data (see the ``synthetic`` package) already resident in HBM; six rotating buffer sets
-(activations, workspace, outputs and weight copies, > 2x the 126 MB L2) keep successive
-steps from hitting in L2. Steps are replayed from a CUDA graph; timing uses CUDA events on
+Default workload: the video-DiT-shaped long sequence (M = 2 x 17550 = 35100 tokens, K=3072,
+N=3072, Kronecker 4x4 (x) 8x8 block transform, per-token centring with the rank-1 restore,
+rank-64 branch), bf16 output: the largest of the five workloads, and it fits one GPU. Inputs are seeded synthetic
+data (see the ``synthetic`` package) already resident in HBM; rotating buffer sets
+(activations, workspace, outputs and weight copies, together > 2x the 126 MB L2) keep
+successive steps from hitting in L2. Steps are replayed from a CUDA graph; timing uses CUDA events on
 the launching stream, max over ranks. For N > 1 every rank runs its own batch (tokens
 are independent: weak scaling, no collective on the data path).
 
@@ -34,7 +35,9 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "W4A4 linear tokens/s; quantize HBM GB/s and GEMM FP4 TFLOPS as % of roofline"
-DEFAULT_WORKLOAD = 2
+DEFAULT_WORKLOAD = 5
+# each phase-isolated timing replays its graph for at least this long
+PHASE_MIN_S = 0.1
 
 
 def _peaks():
@@ -98,7 +101,13 @@ def quantize_comparator(kq, torch, args, w, inp, sets, R, dev) -> dict:
                 fn(j)
         g.replay()
         torch.cuda.synchronize()
-        reps = max(10, min(args.steps, 2000) // R)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        reps = max(10, int(np.ceil(PHASE_MIN_S * 1e3 / max(a.elapsed_time(b), 1e-3))))
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record()
@@ -116,9 +125,9 @@ def quantize_comparator(kq, torch, args, w, inp, sets, R, dev) -> dict:
 
 
 def measured_traffic(kernel: str, workload_label: str):
-    """DRAM bytes per launch of `kernel` from the committed ncu capture
-    (profiles/dram_traffic.json), or None when there is none for this workload or the
-    kernel source has changed since it was taken."""
+    """DRAM bytes per launch of `kernel` (read + write) from the committed ncu capture
+    (profiles/dram_traffic.json) with its note, or None when there is none for this workload
+    or a source file of the kernel has changed since it was taken."""
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
@@ -131,13 +140,16 @@ def measured_traffic(kernel: str, workload_label: str):
                 h.update(f.read())
         if h.hexdigest()[:16] != rec["source_sha256_16"]:
             return None
-        return int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"])
+        return {"bytes": int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"]),
+                "note": rec.get("note", "")}
     except (OSError, ValueError, KeyError):
         return None
 
 
-# nominal dense ratio FP4 : BF16 on B200 (9 : 2.25 PFLOP/s)
+# nominal dense ratio FP4 : BF16 on B200 (9 : 2.25 PFLOP/s), and the nominal dense peaks
 FP4_OVER_BF16 = 4.0
+NOMINAL_FP4_TFLOPS = 9000.0
+NOMINAL_FP16_TFLOPS = 2250.0
 
 
 class Clocks:
@@ -457,21 +469,36 @@ def main():
     if world > 1:
         dist.barrier()
 
-    # per-kernel attribution: the same launches, one phase at a time
-    reps = max(1, min(args.steps, 2000) // R)
+    # per-kernel attribution: the same launches, one phase at a time, each replayed for at
+    # least PHASE_MIN_S of device time whatever --steps is
     if gq is not None:
-        q_ms = timed(gq.replay, reps) / (reps * R)
-        g_ms = timed(gg.replay, reps) / (reps * R)
+        q_fn, g_fn = gq.replay, gg.replay
     else:
-        q_ms = timed(lambda: [kq.quantize_act(L, s["w"], s["X"], s["act"]) for s in sets], reps) / (reps * R)
-        g_ms = timed(lambda: [kq.gemm(L, s["w"], s["act"], w.M, s["Y"], odt) for s in sets], reps) / (reps * R)
+        def q_fn():
+            for s in sets:
+                kq.quantize_act(L, s["w"], s["X"], s["act"])
+
+        def g_fn():
+            for s in sets:
+                kq.gemm(L, s["w"], s["act"], w.M, s["Y"], odt)
+
+    def phase_ms(fn):
+        once = max(timed(fn, 1), 1e-3)
+        reps = max(3, int(np.ceil(PHASE_MIN_S * 1e3 / once)))
+        return timed(fn, reps) / (reps * R), reps
+
+    q_ms, q_reps = phase_ms(q_fn)
+    g_ms, g_reps = phase_ms(g_fn)
     for s in sets:
         assert kq.last_device_error(L, s["act"], w.M) == 0
 
     ms_per_step = elapsed_ms / args.steps
     tokens_per_s = w.M * world * args.steps / (elapsed_ms / 1e3)
 
-    # roofline of the dominant kernel (algorithmic work per launch / event-timed duration)
+    # roofline of the dominant kernel (algorithmic work per launch / event-timed duration).
+    # Each phase is timed alone (graph replays of that phase only), so the denominators are
+    # the burst figures: FP4 = 4 x the measured burst bf16 rate (the nominal 9 : 2.25 dense
+    # ratio), fp16 = the burst bf16 rate, HBM = the measured copy rate.
     peaks = _peaks()
     M, K, N, rp = w.M, w.K, w.N, (64 if w.rank else 0)
     gemm_flops = 2.0 * M * N * K + 2.0 * M * N * w.rank + (M * N if w.center else 0)
@@ -484,26 +511,35 @@ def main():
         gemm_bytes = M * K / 2 + N * K / 2 + (M + N) * K / 32 + M * rp * 2 + N * rp * 2 + N * 4 + \
             (M * 4 if w.center else 0) + ybytes
         q_bytes = M * K * 2 + M * K / 2 + M * K / 32 + M * 4 + M * rp * 2
-    # the contraction's own dtype: FP4 = 4 x the measured bf16 rate; fp16 = the bf16 rate
-    fp4_peak = peaks["bf16_sustained"] * (1.0 if lut else FP4_OVER_BF16)
-    t_tensor = gemm_flops / (fp4_peak * 1e12)
+    tensor_peak = peaks["bf16"] * (1.0 if lut else FP4_OVER_BF16)
+    nominal_peak = NOMINAL_FP16_TFLOPS if lut else NOMINAL_FP4_TFLOPS
+    t_tensor = gemm_flops / (tensor_peak * 1e12)
     t_hbm = gemm_bytes / (peaks["hbm_gbs"] * 1e9)
-    if g_ms >= q_ms:
-        if t_tensor >= t_hbm:
-            ach = gemm_flops / (g_ms * 1e-3) / 1e12
-            roof = {"kernel": "k_gemm_mxf4", "bound": "tensor", "achieved": ach, "peak": fp4_peak,
-                    "unit": "TFLOP/s", "frac": ach / fp4_peak}
-        else:
-            ach = gemm_bytes / (g_ms * 1e-3) / 1e9
-            roof = {"kernel": "k_gemm_mxf4", "bound": "hbm", "achieved": ach,
-                    "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    gname = "k_gemm_mxf4"
+    if t_tensor >= t_hbm:
+        ach = gemm_flops / (g_ms * 1e-3) / 1e12
+        roof_g = {"kernel": gname, "bound": "tensor", "achieved": ach, "peak": tensor_peak,
+                  "unit": "TFLOP/s", "frac": ach / tensor_peak,
+                  "frac_of_nominal": ach / nominal_peak, "nominal_peak": nominal_peak,
+                  "peak_source": peaks["source"] + (" burst bf16 (fp16 rate)" if lut else
+                                                    " burst bf16 x 4 (FP4 rate)")}
     else:
-        ach = q_bytes / (q_ms * 1e-3) / 1e9
-        roof = {"kernel": "k_quantize_rows+k_lowrank_u", "bound": "hbm", "achieved": ach,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
-    roof["traffic"] = measured_traffic(roof["kernel"], w.label)
-    roof["peak_source"] = peaks["source"] + (
-        (" (fp16 = sustained bf16)" if lut else " (FP4 = 4 x sustained bf16)") if roof["unit"] == "TFLOP/s" else "")
+        ach = gemm_bytes / (g_ms * 1e-3) / 1e9
+        roof_g = {"kernel": gname, "bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"],
+                  "unit": "GB/s", "frac": ach / peaks["hbm_gbs"],
+                  "peak_source": peaks["source"] + " copy bandwidth"}
+    roof_g["algorithmic_per_launch"] = gemm_flops if roof_g["unit"] == "TFLOP/s" else gemm_bytes
+    q_ach = q_bytes / (q_ms * 1e-3) / 1e9
+    qname = "k_quantize_rows+k_lowrank_u" if w.rank else "k_quantize_rows"
+    roof_q = {"kernel": qname, "bound": "hbm", "achieved": q_ach, "peak": peaks["hbm_gbs"],
+              "unit": "GB/s", "frac": q_ach / peaks["hbm_gbs"],
+              "peak_source": peaks["source"] + " copy bandwidth", "algorithmic_per_launch": q_bytes}
+    for r_ in (roof_g, roof_q):
+        tr = measured_traffic(r_["kernel"], w.label)
+        r_["traffic"] = tr["bytes"] if tr else None
+        if tr:
+            r_["traffic_note"] = tr["note"]
+    roof = roof_g if g_ms >= q_ms else roof_q
 
     # end-to-end through the host-buffer entry point (pinned memory, copies timed)
     e2e = None
@@ -556,10 +592,14 @@ def main():
                    "l2": f"{R} rotating buffer sets of {set_bytes / 1e6:.0f} MB (> L2)",
                    "graph": graph is not None},
         "phases_ms": {"quantize": q_ms, "gemm": g_ms,
-                      "how": "phase-isolated CUDA-graph replays over the same buffer sets"},
+                      "how": f"phase-isolated CUDA-graph replays over the same buffer sets, "
+                             f"each >= {PHASE_MIN_S * 1e3:.0f} ms ({q_reps} and {g_reps} "
+                             f"replays of {R} launches)"},
         "quantize_gbs": q_bytes / (q_ms * 1e-3) / 1e9,
         "gemm_tflops": gemm_flops / (g_ms * 1e-3) / 1e12,
         "roofline": roof,
+        "roofline_gemm": roof_g,
+        "roofline_quantize": roof_q,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": launches_per_step * args.steps,

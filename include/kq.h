@@ -10,8 +10,9 @@
  *
  * with, prepared once per layer: W' = P^-1 W, W' ~ L1 L2 (rank r, bf16 factors),
  * R = W' - L1 L2 in MXFP4, s = 1^T W, and online U = Xt L1. The low-rank branch runs in
- * 16 bits: U is held as fp16 (saturated at +-65504) and multiplied with L2 (bf16 values,
- * held as fp16) on the tensor cores with fp32 accumulation.
+ * 16 bits: U is held as fp16 (saturated at +-65504, which the device error word reports)
+ * and multiplied with L2 (bf16 values, held as fp16) on the tensor cores with fp32
+ * accumulation.
  *
  * Sources (commentary pages on the methods):
  *   - KroQuant: Kronecker-Structured Block Transforms for Efficient Post-Training
@@ -36,11 +37,11 @@
  *     Buffers must stay alive until that work completes.
  *   - Errors: argument, shape and alignment problems are found on the host and
  *     returned before anything is launched. CUDA launch errors return KQ_ERR_CUDA.
- *     Device-side problems (a bounded wait that ran out) set an error word in the
- *     activation workspace; kq_last_device_error() reports and clears it. Nothing
- *     aborts or traps.
- *   - Alignment: device pointers 256-byte aligned; K % 32 == 0, N % 16 == 0, M >= 1
- *     arbitrary; rank <= 64.
+ *     Device-side problems (a bounded wait that ran out, a low-rank activation outside
+ *     the fp16 range) set bits of an error word in the activation workspace;
+ *     kq_last_device_error() reports and clears it. Nothing aborts or traps.
+ *   - Alignment: device pointers 16-byte aligned (what TMA needs of a global address);
+ *     K % 32 == 0, N % 16 == 0, M >= 1 arbitrary; rank <= 64.
  *   - Determinism: outputs are bitwise reproducible run to run.
  */
 #ifndef KQ_H_
@@ -60,12 +61,15 @@ typedef enum {
   KQ_OK = 0,
   KQ_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum */
   KQ_ERR_UNSUPPORTED_SHAPE = 2,  /* K % 32 != 0, N % 16 != 0, rank > 64, ... */
-  KQ_ERR_ALIGNMENT = 3,          /* a device pointer is not 256-byte aligned */
+  KQ_ERR_ALIGNMENT = 3,          /* a device pointer is not 16-byte aligned */
   KQ_ERR_SINGULAR_TRANSFORM = 4, /* A or B of the Kronecker transform is not invertible */
   KQ_ERR_WORKSPACE_TOO_SMALL = 5,/* a caller buffer is smaller than the size query says */
   KQ_ERR_CUDA = 6,               /* a CUDA runtime/driver/library call failed */
   KQ_ERR_DEVICE_TIMEOUT = 7,     /* a device-side bounded wait ran out (see kq_last_device_error) */
-  KQ_ERR_NO_SM100 = 8            /* the current device is not compute capability 10.0 */
+  KQ_ERR_NO_SM100 = 8,           /* the current device is not compute capability 10.0 */
+  KQ_ERR_LOWRANK_RANGE = 9       /* a low-rank activation U lay outside the fp16 range and was
+                                    saturated at +-65504 (or was not a number); the output
+                                    of that call is not to be trusted */
 } kq_status;
 
 typedef enum { KQ_T_NONE = 0, KQ_T_KRON = 1, KQ_T_RPBH = 2 } kq_transform_kind;
@@ -199,7 +203,7 @@ kq_status kq_quantize_act(const kq_layer_desc *desc, const void *weights, const 
  * Same kernel and pipeline as kq_quantize_act, only the transform differs. The layer
  * descriptor must have no transform, no centring and rank 0 (else KQ_ERR_INVALID_ARG);
  * the matching weights are kq_prepare_weights of diag(s) W for that descriptor.
- * inv_s must be 256-byte aligned. Async on `stream`. */
+ * inv_s must be 16-byte aligned. Async on `stream`. */
 kq_status kq_smooth_quantize_act(const kq_layer_desc *desc, const float *inv_s,
                                  const void *X_bf16, int32_t M, void *act, size_t act_bytes,
                                  kq_stream_t stream);
@@ -238,8 +242,10 @@ kq_status kq_linear_host(const kq_layer_desc *desc, const void *weights, const v
  *     tokens for K = 1152, 9,500 for K = 3072, 2,500 for K = 12288 with a low-rank
  *     branch). Use kq_linear with your own workspace for larger M.
  *   Set-up: the first call made with a given device current looks up the array's
- *     address on that device (cudaGetSymbolAddress) and caches it; later calls only
- *     read the cache. Make that first call before any stream capture begins.
+ *     address on that device (cudaGetSymbolAddress) and caches it with the id of the
+ *     current context; later calls in the same context only read the cache, and a call
+ *     in another context (for example after cudaDeviceReset) looks the address up again.
+ *     Make the first call in a context before any stream capture begins.
  *   Sharing: every call on a device uses the same array, and it keeps what the last
  *     call wrote. Each call clears the error word at its head and rewrites everything
  *     else it reads. Calls whose work can overlap on the GPU (different streams, or
@@ -318,10 +324,22 @@ kq_status kq_debug_encode_f32(const float *V, int32_t M, int32_t K, void *codes,
 kq_status kq_debug_encode_lp_f32(const float *V, int32_t M, int32_t K, double p, void *codes,
                                  void *scales, kq_stream_t stream);
 
-/* Synchronises `stream`, then maps the workspace's device error word to a status
- * (KQ_OK or KQ_ERR_DEVICE_TIMEOUT) and clears it. */
+/* Synchronises `stream`, then maps the workspace's device error word to a status and
+ * clears it: KQ_ERR_DEVICE_TIMEOUT if a bounded device-side wait ran out (it takes
+ * precedence), else KQ_ERR_LOWRANK_RANGE if a low-rank activation was saturated, else
+ * KQ_OK. */
 kq_status kq_last_device_error(const kq_layer_desc *desc, void *act, int32_t M,
                                kq_stream_t stream);
+
+/* Exercises the bounded-wait path without a fault: one warp waits up to limit_us
+ * microseconds (1 .. 1,000,000) on a barrier that nothing completes, records the timeout
+ * in the error word of `act` (kq_act_bytes(desc, M) bytes, device) and returns. The
+ * next kq_last_device_error on that workspace then reports KQ_ERR_DEVICE_TIMEOUT; the
+ * context stays usable. Every wait in the library's kernels is bounded the same way
+ * (2 s), so a pipeline stage that never fills ends the kernel instead of hanging the GPU.
+ * This entry has no counterpart in the method's description. Async on `stream`. */
+kq_status kq_debug_wait_timeout(const kq_layer_desc *desc, void *act, int32_t M,
+                                uint32_t limit_us, kq_stream_t stream);
 
 /* Static string for a status code. */
 const char *kq_status_string(kq_status s);

@@ -85,6 +85,10 @@ def test_null_and_alignment_errors_before_any_launch():
     odd = ctypes.c_void_p(0x1000 + 8)
     ok = ctypes.c_void_p(0x100000)
     assert kq.lib.kq_quantize_act(L.desc, ok, odd, M, ok, 1 << 20, None) == 3
+    # a 16-byte boundary is enough (what a TMA global address needs): the call gets past
+    # the alignment check and stops at the workspace-size check
+    at16 = ctypes.c_void_p(0x1000 + 16)
+    assert kq.lib.kq_quantize_act(L.desc, at16, at16, M, at16, 16, None) == 5
     # too-small workspace
     assert kq.lib.kq_quantize_act(L.desc, ok, ok, M, ok, 16, None) == 5
     # bad output dtype
@@ -112,9 +116,23 @@ def test_lp_entry_points_reject_bad_p():
 
 
 def test_status_strings():
-    for s in range(9):
+    for s in range(10):
         assert kq.status_string(s)
-    assert "timed out" in kq.status_string(7)
+    assert "timed out" in kq.status_string(kq.ERR_DEVICE_TIMEOUT)
+    assert "fp16 range" in kq.status_string(kq.ERR_LOWRANK_RANGE)
+    assert "16-byte" in kq.status_string(3)
+
+
+def test_wait_timeout_entry_validates_before_launch():
+    """The bounded-wait exercise takes a limit of 1 us .. 1 s and an aligned workspace;
+    anything else is refused on the host."""
+    L = kq.Layer(64, 64, 0, False, _kron())
+    ok = ctypes.c_void_p(0x100000)
+    assert kq.lib.kq_debug_wait_timeout(L.desc, ok, 8, 0, None) == 1
+    assert kq.lib.kq_debug_wait_timeout(L.desc, ok, 8, 1000001, None) == 1
+    assert kq.lib.kq_debug_wait_timeout(L.desc, None, 8, 1000, None) == 1
+    assert kq.lib.kq_debug_wait_timeout(L.desc, ok, 0, 1000, None) == 1
+    assert kq.lib.kq_debug_wait_timeout(L.desc, ctypes.c_void_p(0x1000 + 8), 8, 1000, None) == 3
 
 
 def _ln(K, **kw):

@@ -1,11 +1,13 @@
 """GPU: kq_linear_noalloc (the layer on the library's built-in workspace) gives the
 output of kq_linear with a caller-owned workspace, on consecutive calls that reuse the
-built-in workspace with different inputs and sizes, and refuses a token count whose
-workspace would not fit. Named to be collected last, so that it also runs after every
-other GPU test has used the library in the same process."""
+built-in workspace with different inputs and sizes, matches the oracle's layer on its
+own (fp32 output, 1e-3 relative Frobenius), and refuses a token count whose workspace
+would not fit. Named to be collected last, so that it also runs after every other GPU
+test has used the library in the same process."""
 import numpy as np
 import pytest
 
+from oracle import layer as olayer
 from tests.kqtest import cached, make_layer, pack_oracle_weights, rel_fro
 
 pytestmark = pytest.mark.gpu
@@ -48,6 +50,10 @@ def test_noalloc_matches_linear_on_consecutive_calls(cuda_device, index, kw):
             got = _linear(kq, L, wbuf, Xi, out, noalloc=True)
             assert np.all(np.isfinite(got))
             assert rel_fro(got, ref) <= tol
+            if out == kq.OUT_F32:
+                # and on its own against the oracle's fp64 layer
+                Yo = olayer.linear(Xi.cpu(), inp["T"], w.center, prep)
+                assert rel_fro(got, Yo) <= 1e-3
 
 
 def test_noalloc_rejects_too_large_M(cuda_device):

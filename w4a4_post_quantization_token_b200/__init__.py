@@ -18,10 +18,12 @@ __all__ = ["KQError", "Layer", "lib", "library_path", "weights_bytes", "act_byte
            "linear_noalloc", "lloydmax_codebook", "CB_MXFP4", "CB_LLOYDMAX",
            "linear_host", "NOALLOC_WORKSPACE_BYTES",
            "gemm", "weights_pack", "weights_unpack", "act_pack", "act_unpack",
-           "debug_transform", "debug_encode_f32", "last_device_error", "status_string",
+           "debug_transform", "debug_encode_f32", "debug_wait_timeout", "last_device_error",
+           "status_string", "ERR_DEVICE_TIMEOUT", "ERR_LOWRANK_RANGE",
            "OUT_F32", "OUT_BF16", "SYMBOLS"]
 
 OUT_F32, OUT_BF16 = 0, 1
+ERR_DEVICE_TIMEOUT, ERR_LOWRANK_RANGE = 7, 9
 T_NONE, T_KRON, T_RPBH = 0, 1, 2
 _KIND = {"none": T_NONE, "kron": T_KRON, "rpbh": T_RPBH}
 CB_MXFP4, CB_LLOYDMAX = 0, 1
@@ -36,7 +38,7 @@ SYMBOLS = ["kq_weights_bytes", "kq_act_bytes", "kq_prepare_ws_bytes", "kq_prepar
            "kq_weights_unpack", "kq_act_pack", "kq_act_unpack", "kq_debug_transform",
            "kq_debug_encode_f32", "kq_last_device_error", "kq_status_string", "kq_version",
            "kq_linear_noalloc", "kq_smooth_quantize_act", "kq_prepare_weights_lp",
-           "kq_debug_encode_lp_f32", "kq_lloydmax_codebook"]
+           "kq_debug_encode_lp_f32", "kq_lloydmax_codebook", "kq_debug_wait_timeout"]
 
 
 class KQError(RuntimeError):
@@ -94,6 +96,7 @@ _sigs = {
     "kq_debug_transform": (ctypes.c_int, [_D, _P, _P, ctypes.c_int32, _P, _P, _P]),
     "kq_debug_encode_f32": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P, _P]),
     "kq_last_device_error": (ctypes.c_int, [_D, _P, ctypes.c_int32, _P]),
+    "kq_debug_wait_timeout": (ctypes.c_int, [_D, _P, ctypes.c_int32, ctypes.c_uint32, _P]),
     "kq_lloydmax_codebook": (ctypes.c_int, [_P, _P]),
     "kq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "kq_version": (ctypes.c_char_p, []),
@@ -341,5 +344,15 @@ def debug_encode_f32(V, codes, scales, stream=None) -> None:
 
 
 def last_device_error(layer: Layer, act, M: int, stream=None) -> int:
-    """0 if the device error word is clear, else the KQ_ERR_DEVICE_TIMEOUT status."""
+    """0 if the device error word is clear, else ERR_DEVICE_TIMEOUT (a bounded device wait
+    ran out) or ERR_LOWRANK_RANGE (a low-rank activation was saturated to the fp16 range).
+    Synchronises the stream and clears the word."""
     return int(lib.kq_last_device_error(layer.desc, _ptr(act), int(M), _stream(stream)))
+
+
+def debug_wait_timeout(layer: Layer, act, M: int, limit_us: int, stream=None) -> None:
+    """Enqueue one warp that waits limit_us on a barrier nothing completes, so that the
+    next last_device_error on `act` reports ERR_DEVICE_TIMEOUT."""
+    _need(act, __import__("torch").uint8, act_bytes(layer, M), "act")
+    _check(lib.kq_debug_wait_timeout(layer.desc, _ptr(act), int(M), int(limit_us), _stream(stream)),
+           "kq_debug_wait_timeout")

@@ -72,7 +72,9 @@ bool make_tmap(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_
 }
 
 // ---------------------------------------------------------------- validation --------
-bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 255u) == 0; }
+// TMA tensor maps and bulk copies need 16-byte global addresses; every region the library
+// carves out of a caller buffer starts at a 1024-byte multiple from its base
+bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr int kRpbhMaxK = 32736;    // largest K % 32 == 0 with 2 K < 65536
 
@@ -627,12 +629,13 @@ const char* kq_status_string(kq_status s) {
     case KQ_OK: return "ok";
     case KQ_ERR_INVALID_ARG: return "invalid argument";
     case KQ_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
-    case KQ_ERR_ALIGNMENT: return "device pointer not 256-byte aligned";
+    case KQ_ERR_ALIGNMENT: return "device pointer not 16-byte aligned";
     case KQ_ERR_SINGULAR_TRANSFORM: return "Kronecker factor is singular";
     case KQ_ERR_WORKSPACE_TOO_SMALL: return "buffer smaller than the size query";
     case KQ_ERR_CUDA: return "CUDA call failed";
     case KQ_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
     case KQ_ERR_NO_SM100: return "device is not sm_100 (B200)";
+    case KQ_ERR_LOWRANK_RANGE: return "a low-rank activation exceeded the fp16 range (saturated)";
   }
   return "unknown status";
 }
@@ -947,7 +950,24 @@ kq_status kq_last_device_error(const kq_layer_desc* desc, void* act, int32_t M, 
   uint8_t* a = static_cast<uint8_t*>(act);
   if (cudaMemcpy(&word, a + AL.err, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return KQ_ERR_CUDA;
   if (word != 0 && cudaMemset(a + AL.err, 0, 4) != cudaSuccess) return KQ_ERR_CUDA;
+  if (word & KQ_DEV_ERR_TIMEOUT_MASK) return KQ_ERR_DEVICE_TIMEOUT;
+  if (word & KQ_DEV_ERR_U_RANGE) return KQ_ERR_LOWRANK_RANGE;
   return word ? KQ_ERR_DEVICE_TIMEOUT : KQ_OK;
+}
+
+kq_status kq_debug_wait_timeout(const kq_layer_desc* desc, void* act, int32_t M, uint32_t limit_us,
+                                kq_stream_t stream) {
+  kq_status s = check_desc(desc);
+  if (s != KQ_OK) return s;
+  if (!act || M <= 0 || limit_us == 0 || limit_us > 1000000u) return KQ_ERR_INVALID_ARG;
+  if (!aligned(act)) return KQ_ERR_ALIGNMENT;
+  DeviceInfo di;
+  if ((s = current_device(&di)) != KQ_OK) return s;
+  uint32_t* err = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(act) + alayout(desc, M).err);
+  if (launch_wait_never(err, static_cast<uint64_t>(limit_us) * 1000u,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
 }
 
 }  // extern "C"

@@ -165,6 +165,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) k_gemm_mxf4(const __grid_co
           }
         }
       }
+      if (!ok) drain_ring(full, kStages, it);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------- MMA issuer

@@ -102,6 +102,8 @@ cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sm
 cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint8_t* scales,
                               cudaStream_t st, double lp = 0.0);
 cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st);
+// debug: one warp waits limit_ns on a barrier nothing completes, then sets the timeout bit
+cudaError_t launch_wait_never(uint32_t* err, uint64_t limit_ns, cudaStream_t st);
 // LayerNorm front-end, offline: l1gt = diag(gamma) (l1t hi + lo) as hi / lo rows,
 // cg = gamma^T L1', cb = beta^T L1' (float64 sums in fixed order).
 cudaError_t launch_ln_fold(const uint16_t* l1t, const float* gamma, const float* beta, int K,

@@ -572,6 +572,27 @@ __global__ void k_encode_f32(const float* __restrict__ V, int M, int K, uint8_t*
 }
 
 // ----------------------------------------------------------------------------------
+// k_wait_never (debug): one warp waits, with the given limit, on an mbarrier that nothing
+// arrives on. The wait runs out, sets KQ_DEV_ERR_TIMEOUT_FULL in the error word and the
+// kernel returns: the path every kernel's bounded waits take when a stage never fills.
+// ----------------------------------------------------------------------------------
+__global__ void k_wait_never(uint32_t* err, uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(&bar, 0, threadIdx.x == 0 ? err : nullptr, KQ_DEV_ERR_TIMEOUT_FULL, limit_ns);
+  (void)__all_sync(0xffffffffu, ok);
+}
+
+cudaError_t launch_wait_never(uint32_t* err, uint64_t limit_ns, cudaStream_t st) {
+  k_wait_never<<<1, 32, 0, st>>>(err, limit_ns);
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------------
 // k_lowrank_u: U[m, 0..63] = X L1'_hi + X L1'_lo - mu[m] c1, stored as fp16
 // ----------------------------------------------------------------------------------
 // Grid (M/128, S), S in {1, 2, 4, 8}: CTA (mt, ks) accumulates the 128-row tile over its
@@ -593,11 +614,19 @@ constexpr uint32_t kTmemCols = 128;
 static_assert(kSmemBytes == kLowRankSmemBytes, "shared-memory footprint the quantize shape leaves room for");
 }  // namespace lowrank
 
-__device__ __forceinline__ uint32_t f2_to_half2_sat(float a, float b) {
+// fp16 pair of two U values, saturated at +-65504; `over` is set when either lies outside
+// that range or is not a number (the caller reports it through the device error word)
+__device__ __forceinline__ uint32_t f2_to_half2_sat(float a, float b, bool& over) {
+  over |= !(fabsf(a) <= 65504.f) || !(fabsf(b) <= 65504.f);
   a = fminf(fmaxf(a, -65504.f), 65504.f);
   b = fminf(fmaxf(b, -65504.f), 65504.f);
   const __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<const uint32_t*>(&h);
+}
+// one lane of the warp records a saturated U value in the error word
+__device__ __forceinline__ void report_u_range(uint32_t* err, bool over) {
+  if (__any_sync(0xffffffffu, over) && (threadIdx.x & 31) == 0 && err != nullptr)
+    atomicOr(err, KQ_DEV_ERR_U_RANGE);
 }
 
 // One output of the U epilogue from the accumulated x L: acc - mu c1[j], or with the
@@ -637,13 +666,16 @@ __device__ __forceinline__ void lowrank_finish(const LowRankParams& p, const flo
       acc[c] += ld_shared_cluster_f32(mapa_shared(la, static_cast<uint32_t>(src)));
     }
   }
+  bool over = false;
   if (row < p.M) {
     const URowTerms rt = u_row_terms(p, row);
     uint32_t* dst = reinterpret_cast<uint32_t*>(p.u + static_cast<size_t>(row) * kRankPad + j0);
 #pragma unroll
     for (int c = 0; c < kCols; c += 2)
-      dst[c / 2] = f2_to_half2_sat(u_value(p, rt, acc[c], j0 + c), u_value(p, rt, acc[c + 1], j0 + c + 1));
+      dst[c / 2] = f2_to_half2_sat(u_value(p, rt, acc[c], j0 + c), u_value(p, rt, acc[c + 1], j0 + c + 1),
+                                   over);
   }
+  report_u_range(p.err, over);
 }
 
 template <int NS>
@@ -682,19 +714,24 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
   const uint32_t tmem = *tmem_slot;
   grid_dep_launch();
 
+  bool loads_ok = true;              // warp 0: every issued load was taken by the MMA warp
   if (warp == 0) {
     if (lane == 0) {
-      for (int i = 0; i < nk; ++i) {
+      int i = 0;
+      for (; i < nk; ++i) {
         const int s = i % kStages;
         if (i >= kStages &&
-            !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, p.err, KQ_DEV_ERR_TIMEOUT_EMPTY))
+            !mbar_wait(&empty[s], ((i / kStages) - 1) & 1, p.err, KQ_DEV_ERR_TIMEOUT_EMPTY)) {
+          loads_ok = false;
           break;
+        }
         uint8_t* a = stage0 + s * kStageBytes;
         mbar_arrive_expect_tx(&full[s], kStageBytes);
         const int kc = i * S + ks;
         tma_load_2d(a, &p.tmap_x, kc * kChunkK, m0, &full[s]);
         tma_load_2d(a + kABytes, &p.tmap_l1, kc * kChunkK, 0, &full[s]);
       }
+      if (!loads_ok) drain_ring(full, kStages, i);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -739,22 +776,28 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
     }
     if (S == 1) {
       const int row = m0 + rl;
+      bool over = false;
       if (ok && row < p.M) {
         const URowTerms rt = u_row_terms(p, row);
         uint32_t packed[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          packed[j] = f2_to_half2_sat(u_value(p, rt, u[2 * j], 2 * j), u_value(p, rt, u[2 * j + 1], 2 * j + 1));
+          packed[j] = f2_to_half2_sat(u_value(p, rt, u[2 * j], 2 * j), u_value(p, rt, u[2 * j + 1], 2 * j + 1),
+                                      over);
         uint4* dst = reinterpret_cast<uint4*>(p.u + static_cast<size_t>(row) * kRankPad);
 #pragma unroll
         for (int v = 0; v < 8; ++v)
           dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
       }
-    } else {
+      report_u_range(p.err, over);
+    } else if (ok) {
+      // (after a wait ran out, loads may still land in the ring that `part` overlays: the
+      // partials are left alone and the call reports the timeout)
 #pragma unroll
       for (int j = 0; j < 64; ++j) part[j * 128 + rl] = u[j];   // column-major: conflict-free
     }
   }
+  (void)loads_ok;
   if (S > 1) {
     __syncwarp();
     cluster_sync();                       // every partial is in place

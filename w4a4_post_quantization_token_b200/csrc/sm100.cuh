@@ -18,7 +18,10 @@ enum : uint32_t {
   KQ_DEV_ERR_TIMEOUT_EMPTY = 1u << 1,  // producer gave up waiting for a free stage
   KQ_DEV_ERR_TIMEOUT_ACC = 1u << 2,    // epilogue gave up waiting for the accumulator
   KQ_DEV_ERR_BAD_TMEM = 1u << 3,       // TMEM allocation returned an unexpected address
+  KQ_DEV_ERR_U_RANGE = 1u << 8,        // a low-rank activation was outside the fp16 range
 };
+// bits that report a wait that ran out (KQ_ERR_DEVICE_TIMEOUT)
+constexpr uint32_t KQ_DEV_ERR_TIMEOUT_MASK = 0xFFu;
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s per wait
 
@@ -56,19 +59,28 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait until the barrier's phase with the given parity has completed.
-// Returns false (and sets `code` in *err) if it did not within kWaitLimitNs.
+// Returns false (and sets `code` in *err) if it did not within limit_ns.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* err,
-                                          uint32_t code) {
+                                          uint32_t code, uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(a, parity)) return true;
-    if ((i & 255u) == 0u && globaltimer_ns() - t0 > kWaitLimitNs) {
+    if ((i & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) {
       if (err) atomicOr(err, code);
       return false;
     }
   }
+}
+
+// After a producer stopped early (a wait ran out), wait -- bounded, without reporting --
+// for the loads it issued that no consumer has taken: the last min(issued, stages) ring
+// slots, load j into slot j % stages completing that slot's phase j / stages. No TMA
+// write may still be landing in shared memory when the CTA exits.
+__device__ __forceinline__ void drain_ring(uint64_t* full, int stages, int64_t issued) {
+  for (int64_t j = issued > stages ? issued - stages : 0; j < issued; ++j)
+    mbar_wait(&full[j % stages], static_cast<uint32_t>(j / stages) & 1u, nullptr, 0u);
 }
 
 // ------------------------------- TMA -------------------------------------------
