@@ -25,6 +25,13 @@ CASES = [  # (workload law, overrides): ragged M, every transform, centring on/o
     (5, dict(M=129, N=256, rank=64)),
     (1, dict(M=33, center=False, K=64, N=64, rank=0)),
     (2, dict(M=50, center=True, K=2048, N=128, rank=5)),
+    # the streaming Kronecker path: K % 64 == 32 (a half piece), centring with rank 0 (the
+    # statistics alone), a low-rank branch without centring, several row tiles at S = 1
+    (1, dict(M=45, K=96, N=64, rank=4)),
+    (3, dict(M=140, K=160, N=64, rank=8)),
+    (5, dict(M=77, N=64, rank=0)),
+    (1, dict(M=260, center=False, rank=16)),
+    (3, dict(M=1300, K=3072, N=64, rank=32)),
 ]
 
 

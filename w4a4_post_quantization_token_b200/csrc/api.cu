@@ -416,8 +416,103 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   return KQ_OK;
 }
 
+// Layers whose transform is Kronecker or none, without the LayerNorm front-end or the
+// codebook, take the streaming path: k_lowrank_u forms U and (centring) the token means from
+// 128-row x 64-element pieces of X, then k_quantize_chunks centres, transforms and encodes
+// the same pieces. The other layers (RPBH's global gather, the front-end's statistics, the
+// codebook's sigma) stage whole token rows in k_quantize_rows.
+bool chunk_path(const kq_layer_desc* d) {
+  return (d->t.kind == KQ_T_KRON || d->t.kind == KQ_T_NONE) && d->ln.on == 0 &&
+         d->codebook == KQ_CB_MXFP4;
+}
+
+void kron_pairs(const kq_layer_desc* d, uint64_t* Ap, uint64_t* Bp) {
+  auto pair = [](float lo, float hi) {
+    uint32_t a, b;
+    std::memcpy(&a, &lo, 4);
+    std::memcpy(&b, &hi, 4);
+    return (static_cast<uint64_t>(b) << 32) | a;
+  };
+  for (int i = 0; i < 4; ++i)
+    for (int k = 0; k < 4; ++k) Ap[4 * i + k] = pair(d->t.A[4 * i + k], d->t.A[4 * i + k]);
+  for (int j = 0; j < 8; ++j)
+    for (int l = 0; l < 4; ++l) Bp[4 * j + l] = pair(d->t.B[8 * j + 2 * l], d->t.B[8 * j + 2 * l + 1]);
+}
+
+// The streaming path. act == nullptr is the debug launch: Xt [M, K] and mu [M] are written
+// instead of the workspace (the means' rounding remainders are parked in Xt[row][0] until
+// the quantize kernel overwrites that row).
+kq_status run_chunk_path(const kq_layer_desc* d, const void* weights, const void* X, int M,
+                         uint8_t* act, float* xt, float* mu_dbg, cudaStream_t st,
+                         const DeviceInfo& di, bool keep_err) {
+  const WeightsLayout WL = wlayout(d);
+  const ActLayout AL = alayout(d, M);
+  const bool debug = act == nullptr;
+  const bool center = d->center != 0;
+  const bool lr = d->rank > 0 && !debug;
+  const int K = d->K;
+  ChunkParams cp;
+  std::memset(&cp, 0, sizeof(cp));
+  if (!make_tmap(&cp.tmap_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, static_cast<uint64_t>(K),
+                 static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, 64, 128,
+                 CU_TENSOR_MAP_SWIZZLE_128B))
+    return KQ_ERR_CUDA;
+  if (d->t.kind == KQ_T_KRON) kron_pairs(d, cp.Ap, cp.Bp);
+  cp.M = M; cp.K = K;
+  cp.m_pad = static_cast<int>(AL.m_pad);
+  cp.tiles = static_cast<int>(cdiv(M, 128));
+  cp.pairs = static_cast<int>(cdiv(K, 128));
+  cp.katoms = sf_katoms(K);
+  uint32_t* err = debug ? nullptr : reinterpret_cast<uint32_t*>(act + AL.err);
+  float* mu = debug ? mu_dbg : reinterpret_cast<float*>(act + AL.mu);
+  float* mulo = debug ? xt : reinterpret_cast<float*>(act + AL.mulo);
+  const int64_t mulo_stride = debug ? K : 1;
+  bool first = true;
+  if (center || lr) {
+    LowRankParams lp;
+    std::memset(&lp, 0, sizeof(lp));
+    lp.tmap_x = cp.tmap_x;
+    if (lr) {
+      const uint8_t* w = static_cast<const uint8_t*>(weights);
+      if (!make_tmap(&lp.tmap_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w + WL.l1t, static_cast<uint64_t>(K),
+                     kUCols, static_cast<uint64_t>(K) * 2, 64, kUCols, CU_TENSOR_MAP_SWIZZLE_128B))
+        return KQ_ERR_CUDA;
+      lp.c1 = reinterpret_cast<const float*>(w + WL.c1);
+      lp.u = reinterpret_cast<uint16_t*>(act + AL.u);
+    }
+    lp.lowrank = lr ? 1 : 0;
+    lp.stats = center ? 1 : 0;
+    lp.clear_err = (!debug && !keep_err) ? 1 : 0;
+    lp.m_pad = debug ? M : static_cast<int>(AL.m_pad);
+    lp.mu_out = mu;
+    lp.mulo_out = mulo;
+    lp.mulo_stride = mulo_stride;
+    lp.M = M; lp.K = K; lp.split = u_split(M, K);
+    lp.deep = 1;                         // alone on its SMs: the deep ring
+    lp.err = err;
+    if (launch_lowrank_u(lp, st, /*dependent=*/false) != cudaSuccess) return KQ_ERR_CUDA;
+    first = false;
+  } else if (debug) {
+    if (cudaMemsetAsync(mu_dbg, 0, static_cast<size_t>(M) * 4, st) != cudaSuccess) return KQ_ERR_CUDA;
+  }
+  cp.clear_err = (first && !debug && !keep_err) ? 1 : 0;
+  cp.mu = center ? mu : nullptr;
+  cp.mulo = center ? mulo : nullptr;
+  cp.mulo_stride = mulo_stride;
+  cp.mu_clear = (center || debug) ? nullptr : reinterpret_cast<float*>(act + AL.mu);
+  cp.codes = debug ? nullptr : act + AL.codes;
+  cp.sf = debug ? nullptr : act + AL.sf;
+  cp.xt = debug ? xt : nullptr;
+  cp.err = err;
+  if (launch_quantize_chunks(cp, d->t.kind == KQ_T_KRON ? 1 : 0, center, debug, !first, di.sms, st) !=
+      cudaSuccess)
+    return KQ_ERR_CUDA;
+  return KQ_OK;
+}
+
 kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* X, int M,
                        uint8_t* act, cudaStream_t st, const DeviceInfo& di, bool keep_err = false) {
+  if (chunk_path(d)) return run_chunk_path(d, weights, X, M, act, nullptr, nullptr, st, di, keep_err);
   const WeightsLayout WL = wlayout(d);
   const ActLayout AL = alayout(d, M);
   QuantParams qp;
@@ -446,6 +541,8 @@ kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* 
       lp.lnm = reinterpret_cast<const float*>(act + AL.lnm);
       lp.lnr = reinterpret_cast<const float*>(act + AL.lnr);
     }
+    lp.lowrank = 1;
+    lp.stats = 0;                        // the means come from the quantize kernel
     lp.mu = d->center ? reinterpret_cast<const float*>(act + AL.mu) : nullptr;
     lp.u = reinterpret_cast<uint16_t*>(act + AL.u);
     lp.M = M; lp.K = d->K; lp.split = u_split(M, d->K);
@@ -894,6 +991,9 @@ kq_status kq_debug_transform(const kq_layer_desc* desc, const void* weights, con
   if (!aligned(X_bf16) || !aligned(Xt) || !aligned(weights)) return KQ_ERR_ALIGNMENT;
   DeviceInfo di;
   if ((s = current_device(&di)) != KQ_OK) return s;
+  if (chunk_path(desc))
+    return run_chunk_path(desc, weights, X_bf16, M, nullptr, Xt, mu, reinterpret_cast<cudaStream_t>(stream),
+                          di, false);
   QuantParams qp;
   s = fill_quant_params(desc, weights, X_bf16, M, nullptr, &qp, di);
   if (s != KQ_OK) return s;

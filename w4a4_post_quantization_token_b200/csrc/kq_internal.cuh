@@ -65,8 +65,16 @@ struct QuantParams {
 struct LowRankParams {
   CUtensorMap tmap_x;          // X [M, K] bf16, box 64 x 128, 128-byte swizzle
   CUtensorMap tmap_l1;         // [kUCols, K] bf16, box 64 x kUCols, 128-byte swizzle
+  int lowrank;                 // 1: U = X L1' - mu c1 (rank > 0); 0: statistics only
+  int stats;                   // 1: form the token means from the streamed X (centring) and
+                               //    write them; 0: read them from `mu` (or none)
+  int clear_err;               // first kernel of the call: clear the device error word
+  int m_pad;                   // rows of the padded workspace (mu_out is zeroed up to it)
+  float* mu_out;               // stats: fp32(mu) [m_pad]
+  float* mulo_out;             // stats: fp32(mu - fp32(mu)) for rows < M, at row * mulo_stride
+  int64_t mulo_stride;
   const float* c1;             // [64]
-  const float* mu;             // [M] token means (null without centring)
+  const float* mu;             // [M] token means (null without centring, unused with stats)
   uint16_t* u;                 // U [M, 64] fp16
   int deep;                    // 1: the quantize CTAs leave no room on the SM, use the deep ring
   int ln;                      // LayerNorm front-end: L1 map is diag(gamma) L1', and
@@ -75,6 +83,27 @@ struct LowRankParams {
   const float* lnm;            //   per-token m and rstd from the quantize kernel
   const float* lnr;
   int M, K, split;             // split: CTAs (one cluster) per 128-row tile, 1/2/4/8
+  uint32_t* err;
+};
+
+// k_quantize_chunks: the online half for the Kronecker transform (or none) on 128-row x
+// 64-element pieces of X, with the token means already formed by k_lowrank_u (stats).
+struct ChunkParams {
+  CUtensorMap tmap_x;          // X [M, K] bf16, box 64 x 128, 128-byte swizzle
+  uint64_t Ap[16];             // Kronecker A as pairs (A[i][k], A[i][k]), index 4 i + k
+  uint64_t Bp[32];             // Kronecker B as pairs (B[j][2l], B[j][2l+1]), index 4 j + l
+  int M, K, m_pad;
+  int tiles;                   // cdiv(M, 128)
+  int pairs;                   // pieces of 4 blocks per row: cdiv(K, 128)
+  int clear_err;               // first kernel of the call: clear the device error word
+  int64_t katoms;
+  const float* mu;             // centring: fp32(mu) [M]
+  const float* mulo;           // centring: fp32(mu - fp32(mu)), row r at r * mulo_stride
+  int64_t mulo_stride;
+  float* mu_clear;             // no centring: the workspace's means [m_pad], set to 0 here
+  uint8_t* codes;              // act codes [M, K/2]
+  uint8_t* sf;                 // act scales (tensor-core layout, rows padded to m_pad)
+  float* xt;                   // debug: transformed values [M, K] instead of codes / scales
   uint32_t* err;
 };
 
@@ -101,7 +130,11 @@ cudaError_t launch_quantize_rows(const QuantParams& p, bool debug_xt, int num_sm
                                  cudaStream_t st);
 cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint8_t* scales,
                               cudaStream_t st, double lp = 0.0);
-cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st);
+cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st, bool dependent = true);
+// kind: 0 none, 1 Kronecker; dependent: launched as a programmatic dependent of the previous
+// kernel in the stream (the statistics kernel)
+cudaError_t launch_quantize_chunks(const ChunkParams& p, int kind, bool center, bool debug_xt,
+                                   bool dependent, int num_sms, cudaStream_t st);
 // debug: one warp waits limit_ns on a barrier nothing completes, then sets the timeout bit
 cudaError_t launch_wait_never(uint32_t* err, uint64_t limit_ns, cudaStream_t st);
 // LayerNorm front-end, offline: l1gt = diag(gamma) (l1t hi + lo) as hi / lo rows,

@@ -133,6 +133,7 @@ struct ActLayout {
   size_t codes = 0;    // uint8 [M, K/2] (MXFP4) or fp16 [M, K] (Lloyd-Max operand)
   size_t sf = 0;       // uint8 tiled, rows padded to 128 (MXFP4 only)
   size_t mu = 0;       // f32 [m_pad]
+  size_t mulo = 0;     // f32 [m_pad] fp32(mu - fp32(mu)) (Kronecker / no-transform path)
   size_t u = 0;        // fp16 [M, rp]
   size_t lnm = 0;      // f32 [m_pad] LayerNorm mean of x (front-end on)
   size_t lnr = 0;      // f32 [m_pad] LayerNorm 1/sqrt(v + eps)
@@ -149,6 +150,7 @@ struct ActLayout {
     L.codes = o;  o = align_up(o + static_cast<size_t>(M) * (lut ? K * 2 : K / 2), kAlign);
     L.sf = o;     o = align_up(o + (lut ? 0 : sf_bytes(L.m_pad, K)), kAlign);
     L.mu = o;     o = align_up(o + static_cast<size_t>(L.m_pad) * 4, kAlign);
+    L.mulo = o;   o = align_up(o + static_cast<size_t>(L.m_pad) * 4, kAlign);
     L.u = o;      o = align_up(o + static_cast<size_t>(M) * L.rp * 2, kAlign);
     L.lnm = o;    o = align_up(o + (ln ? static_cast<size_t>(L.m_pad) * 4 : 0), kAlign);
     L.lnr = o;    o = align_up(o + (ln ? static_cast<size_t>(L.m_pad) * 4 : 0), kAlign);

@@ -631,11 +631,12 @@ __device__ __forceinline__ void report_u_range(uint32_t* err, bool over) {
 
 // One output of the U epilogue from the accumulated x L: acc - mu c1[j], or with the
 // LayerNorm front-end (L = diag(gamma) L1') rstd acc - rstd m cg[j] + cb[j] - mu c1[j],
-// which is y L1' - mean(y) c1 for y = LayerNorm(x).
+// which is y L1' - mean(y) c1 for y = LayerNorm(x). mu is the row's fp32 mean (0 when the
+// layer does not centre).
 struct URowTerms { float mu, rs, rm; };
-__device__ __forceinline__ URowTerms u_row_terms(const LowRankParams& p, int row) {
+__device__ __forceinline__ URowTerms u_row_terms(const LowRankParams& p, int row, float mu) {
   URowTerms t;
-  t.mu = (p.mu != nullptr) ? p.mu[row] : 0.f;
+  t.mu = mu;
   t.rs = p.ln ? p.lnr[row] : 1.f;
   t.rm = p.ln ? t.rs * p.lnm[row] : 0.f;
   return t;
@@ -645,16 +646,65 @@ __device__ __forceinline__ float u_value(const LowRankParams& p, const URowTerms
   return acc - t.mu * p.c1[j];
 }
 
-// Cluster reduction of the S fp32 partials ([64][128] column-major in each CTA's smem):
-// CTA ks finalises rows [ks*128/S, (ks+1)*128/S); S threads per row, 64/S columns each,
-// summed over the source CTAs in rank order.
+// Sum of the 64 bf16 values of one staged row piece (128 bytes, 128-byte swizzle, row rl of
+// the tile): fp32 within each 32-element block (pairs, then the two halves), the two block
+// sums added in float64.
+__device__ __forceinline__ double chunk_row_sum(const uint8_t* tile, int rl) {
+  const uint8_t* rowp = tile + static_cast<uint32_t>(rl) * 128u;
+  double s = 0.0;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint64_t acc = 0;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 q = *reinterpret_cast<const uint4*>(
+          rowp + 16u * ((static_cast<uint32_t>(4 * h + c)) ^ (static_cast<uint32_t>(rl) & 7u)));
+      const uint64_t s0 = fadd2(bf16x2_to_f2(q.x), bf16x2_to_f2(q.y));
+      const uint64_t s1 = fadd2(bf16x2_to_f2(q.z), bf16x2_to_f2(q.w));
+      acc = c == 0 ? fadd2(s0, s1) : fadd2(acc, fadd2(s0, s1));
+    }
+    s += static_cast<double>(f2lo(acc) + f2hi(acc));
+  }
+  return s;
+}
+
+// The row mean as written for the rest of the layer: fp32(mu) for every row of the padded
+// workspace (0 beyond M), and the rounding remainder fp32(mu - fp32(mu)) for rows < M.
+__device__ __forceinline__ float write_row_mean(const LowRankParams& p, int row, double mu64) {
+  const float mh = static_cast<float>(mu64);
+  if (row < p.M) {
+    p.mu_out[row] = mh;
+    p.mulo_out[static_cast<int64_t>(row) * p.mulo_stride] = static_cast<float>(mu64 - static_cast<double>(mh));
+  } else if (row < p.m_pad) {
+    p.mu_out[row] = 0.f;
+  }
+  return mh;
+}
+
+// Cluster reduction of the S partials: the fp32 U partials ([64][128] column-major in each
+// CTA's smem) and, for the statistics, the float64 row sums (psum[128]). CTA ks finalises
+// rows [ks*128/S, (ks+1)*128/S); S threads per row, 64/S columns each, summed over the
+// source CTAs in rank order (deterministic). Every thread of a row forms the same mean.
 template <int S>
-__device__ __forceinline__ void lowrank_finish(const LowRankParams& p, const float* part, int m0,
-                                               int ks, int t) {
+__device__ __forceinline__ void lowrank_finish(const LowRankParams& p, const float* part,
+                                               const double* psum, int m0, int ks, int t) {
   constexpr int kRows = 128 / S, kCols = 64 / S;
   const int rl = ks * kRows + t % kRows;
   const int j0 = (t / kRows) * kCols;
   const int row = m0 + rl;
+  float mu = 0.f;
+  if (p.stats) {
+    double sum = 0.0;
+#pragma unroll
+    for (int src = 0; src < S; ++src)
+      sum += ld_shared_cluster_f64(mapa_shared(smem_u32(psum + rl), static_cast<uint32_t>(src)));
+    const double mu64 = sum / static_cast<double>(p.K);
+    mu = static_cast<float>(mu64);
+    if (j0 == 0) write_row_mean(p, row, mu64);
+  } else if (p.mu != nullptr && row < p.M) {
+    mu = p.mu[row];
+  }
+  if (!p.lowrank) return;
   float acc[kCols];
 #pragma unroll
   for (int c = 0; c < kCols; ++c) acc[c] = 0.f;
@@ -668,7 +718,7 @@ __device__ __forceinline__ void lowrank_finish(const LowRankParams& p, const flo
   }
   bool over = false;
   if (row < p.M) {
-    const URowTerms rt = u_row_terms(p, row);
+    const URowTerms rt = u_row_terms(p, row, mu);
     uint32_t* dst = reinterpret_cast<uint32_t*>(p.u + static_cast<size_t>(row) * kRankPad + j0);
 #pragma unroll
     for (int c = 0; c < kCols; c += 2)
@@ -678,6 +728,10 @@ __device__ __forceinline__ void lowrank_finish(const LowRankParams& p, const flo
   report_u_range(p.err, over);
 }
 
+// Warps: 0 TMA producer, 1 TMEM allocator and MMA issuer, 2..5 epilogue (thread = tile row).
+// With `stats` the epilogue warps also sum each staged row piece as it lands (before the
+// stage is released), which gives the token means of a centred layer from the same read of
+// X; with `lowrank` off only that part runs (no L1' stream, no TMEM, no MMA).
 template <int NS>
 __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ LowRankParams p) {
   using namespace lowrank;
@@ -691,32 +745,40 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
   uint8_t* stage0 = smem + 1024;
   float* part = reinterpret_cast<float*>(stage0);   // [64][128] after the main loop (S > 1)
+  double* psum = reinterpret_cast<double*>(stage0 + kStages * kStageBytes);   // [128] (S > 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int mt = blockIdx.x, ks = blockIdx.y, S = gridDim.y;
   const int m0 = mt * kTileM;
   const int KT = static_cast<int>(cdiv(p.K, kChunkK));
+  const bool lr = p.lowrank != 0, stats = p.stats != 0;
   // the S CTAs of a row tile take the 64-element K chunks in turn (chunk i S + ks), so
   // that at any time they read neighbouring 128-byte pieces of the same rows
   const int nk = KT > ks ? (KT - ks + S - 1) / S : 0;
+  // first kernel of a call: clear the device error word (see k_quantize_rows)
+  if (p.clear_err && mt == 0 && ks == 0 && threadIdx.x == 0 && p.err != nullptr) *p.err = 0u;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], (lr ? 1 : 0) + (stats ? 4 : 0));   // MMA commit, epilogue warps
+    }
     mbar_init(accf, 1);
     fence_mbar_init();
     prefetch_tmap(&p.tmap_x);
-    prefetch_tmap(&p.tmap_l1);
+    if (lr) prefetch_tmap(&p.tmap_l1);
   }
-  if (warp == 1) { tmem_alloc(tmem_slot, kTmemCols); tmem_relinquish(); }
+  if (lr && warp == 1) { tmem_alloc(tmem_slot, kTmemCols); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = lr ? *tmem_slot : 0u;
   grid_dep_launch();
 
-  bool loads_ok = true;              // warp 0: every issued load was taken by the MMA warp
   if (warp == 0) {
     if (lane == 0) {
+      bool loads_ok = true;            // every issued load was taken by its consumers
+      const uint32_t bytes = lr ? kStageBytes : kABytes;
       int i = 0;
       for (; i < nk; ++i) {
         const int s = i % kStages;
@@ -726,15 +788,15 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
           break;
         }
         uint8_t* a = stage0 + s * kStageBytes;
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        mbar_arrive_expect_tx(&full[s], bytes);
         const int kc = i * S + ks;
         tma_load_2d(a, &p.tmap_x, kc * kChunkK, m0, &full[s]);
-        tma_load_2d(a + kABytes, &p.tmap_l1, kc * kChunkK, 0, &full[s]);
+        if (lr) tma_load_2d(a + kABytes, &p.tmap_l1, kc * kChunkK, 0, &full[s]);
       }
       if (!loads_ok) drain_ring(full, kStages, i);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
+    if (lr && lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(kTileM, kUCols);
       for (int i = 0; i < nk; ++i) {
         const int s = i % kStages;
@@ -754,31 +816,49 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
     // epilogue warps 2..5: TMEM lane quadrant = warp % 4; thread owns tile row rl
     const int q = warp & 3;
     const int rl = 32 * q + lane;
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, p.err, KQ_DEV_ERR_TIMEOUT_ACC));
-    // the token means come from the quantize grid launched just before this one; every CTA
-    // also waits for it before exiting, so the GEMM's wait on this grid covers both
+    const int row = m0 + rl;
+    bool ok = true;
+    double rsum = 0.0;
+    if (stats) {
+      for (int i = 0; i < nk; ++i) {
+        const int s = i % kStages;
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (i / kStages) & 1, p.err, KQ_DEV_ERR_TIMEOUT_FULL));
+        if (!ok) break;
+        rsum += chunk_row_sum(stage0 + s * kStageBytes, rl);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+    }
+    if (lr) ok = __all_sync(0xffffffffu, mbar_wait(accf, 0, p.err, KQ_DEV_ERR_TIMEOUT_ACC) && ok);
+    // without the statistics the token means come from the quantize grid launched just
+    // before this one; every CTA also waits for the preceding grid before exiting, so the
+    // GEMM's wait on this grid covers both
     grid_dep_wait();
     tc_fence_after();
-    const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
     float u[64];
+    if (lr) {
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t hi[32], lo[32];
-      tmem_ld_32x32b_x32(tbase + 32 * h, hi);
-      tmem_ld_32x32b_x32(tbase + 64 + 32 * h, lo);
-      tmem_ld_wait();
+      for (int h = 0; h < 2; ++h) {
+        uint32_t hi[32], lo[32];
+        tmem_ld_32x32b_x32(tbase + 32 * h, hi);
+        tmem_ld_32x32b_x32(tbase + 64 + 32 * h, lo);
+        tmem_ld_wait();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) u[32 * h + j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+        for (int j = 0; j < 32; ++j) u[32 * h + j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+      }
     }
-    if (!ok || nk == 0) {
+    if (!ok || nk == 0 || !lr) {
 #pragma unroll
       for (int j = 0; j < 64; ++j) u[j] = 0.f;
     }
     if (S == 1) {
-      const int row = m0 + rl;
+      float mu = 0.f;
+      if (stats) mu = ok ? write_row_mean(p, row, rsum / static_cast<double>(p.K)) : 0.f;
+      else if (p.mu != nullptr && row < p.M) mu = p.mu[row];
       bool over = false;
-      if (ok && row < p.M) {
-        const URowTerms rt = u_row_terms(p, row);
+      if (lr && ok && row < p.M) {
+        const URowTerms rt = u_row_terms(p, row, mu);
         uint32_t packed[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j)
@@ -793,28 +873,240 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
     } else if (ok) {
       // (after a wait ran out, loads may still land in the ring that `part` overlays: the
       // partials are left alone and the call reports the timeout)
+      if (lr) {
 #pragma unroll
-      for (int j = 0; j < 64; ++j) part[j * 128 + rl] = u[j];   // column-major: conflict-free
+        for (int j = 0; j < 64; ++j) part[j * 128 + rl] = u[j];   // column-major: conflict-free
+      }
+      if (stats) psum[rl] = rsum;
     }
   }
-  (void)loads_ok;
   if (S > 1) {
     __syncwarp();
     cluster_sync();                       // every partial is in place
     if (warp >= 2) {
-      if (S == 2) lowrank_finish<2>(p, part, m0, ks, threadIdx.x - 64);
-      else if (S == 4) lowrank_finish<4>(p, part, m0, ks, threadIdx.x - 64);
-      else lowrank_finish<8>(p, part, m0, ks, threadIdx.x - 64);
+      if (S == 2) lowrank_finish<2>(p, part, psum, m0, ks, threadIdx.x - 64);
+      else if (S == 4) lowrank_finish<4>(p, part, psum, m0, ks, threadIdx.x - 64);
+      else lowrank_finish<8>(p, part, psum, m0, ks, threadIdx.x - 64);
     }
     __syncwarp();
     cluster_sync();                       // no CTA leaves while others still read its smem
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (lr && warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// ----------------------------------------------------------------------------------
+// k_quantize_chunks: centring, Kronecker block transform (or none) and MXFP4 encoding on
+// 128-row x 64-element pieces of X
+// ----------------------------------------------------------------------------------
+// The token means are formed beforehand from the same 128 x 64 pieces (k_lowrank_u with
+// stats, which also produces U), so no whole token row has to be staged here: X streams
+// through a ring of pieces (TMA, 128-byte swizzle, row r of a piece at byte 128 r, its
+// 16-byte chunk c at c ^ (r % 8)), and a thread owns one row of a piece at a time.
+//
+// Work items are (row tile, pair of pieces) = 128 rows x 4 blocks, walked from the last row
+// tile to the first: run after the statistics kernel, the first items re-read the rows that
+// kernel read last, which are still in L2. CTA c takes a contiguous range of items.
+// Warps: 0 TMA producer; 1..12 three groups of four consumer warps (thread = tile row),
+// group g taking every third item of the CTA's range. Per item a thread centres, transforms
+// and encodes its row's 4 blocks, writes 64 bytes of codes and one 32-bit scale word.
+namespace chunkq {
+constexpr int kStages = 8;
+constexpr int kGroups = 3;
+constexpr int kThreads = 32 * (1 + 4 * kGroups);
+constexpr uint32_t kStageBytes = 128 * 128;             // 128 rows x 64 bf16
+constexpr uint32_t kSmemBytes = 1024 + kStages * kStageBytes + 1024;
+}  // namespace chunkq
+
+template <int KIND, int CENTER, bool DEBUG_XT>
+__global__ void __launch_bounds__(chunkq::kThreads, 1) k_quantize_chunks(const __grid_constant__ ChunkParams p) {
+  using namespace chunkq;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(align_up(reinterpret_cast<uintptr_t>(smem_raw), 1024));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kStages;
+  uint8_t* stage0 = smem + 1024;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nb = p.K / kBlock;
+  const int KC = static_cast<int>(cdiv(p.K, 64));
+  const int PP = p.pairs;
+  const int nb_pad = static_cast<int>(p.katoms) * 4;
+  const int64_t T = static_cast<int64_t>(p.tiles) * PP;
+  const int64_t G = gridDim.x;
+  const int64_t q0 = T * blockIdx.x / G, q1 = T * (blockIdx.x + 1) / G;
+
+  if (p.clear_err && blockIdx.x == 0 && threadIdx.x == 0 && p.err != nullptr) *p.err = 0u;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 4); }
+    fence_mbar_init();
+    prefetch_tmap(&p.tmap_x);
+  }
+  __syncthreads();
+  grid_dep_launch();                       // the GEMM may start its prologue
+
+  if (warp == 0) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      int64_t n = 0;
+      bool ok = true;
+      for (int64_t q = q0; q < q1 && ok; ++q) {
+        const int tile = p.tiles - 1 - static_cast<int>(q / PP);
+        const int pair = static_cast<int>(q % PP);
+        for (int cc = 0; cc < 2; ++cc, ++n) {
+          const int s = static_cast<int>(n % kStages);
+          if (n >= kStages &&
+              !mbar_wait(&empty[s], static_cast<uint32_t>(n / kStages - 1) & 1u, p.err,
+                         KQ_DEV_ERR_TIMEOUT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const int chunk = 2 * pair + cc;
+          if (chunk < KC) {
+            mbar_arrive_expect_tx(&full[s], kStageBytes);
+            tma_load_2d(stage0 + s * kStageBytes, &p.tmap_x, chunk * 64, tile * 128, &full[s]);
+          } else {
+            mbar_arrive(&full[s]);         // K % 128 == 64: the pair's second piece is empty
+          }
+        }
+      }
+      if (!ok) drain_ring(full, kStages, n);
+    }
+  } else {
+    // ------------------------------------------------------------- consumers
+    const int cw = warp - 1;
+    const int g = cw >> 2;
+    const int rl = 32 * (cw & 3) + lane;
+    // the means come from the statistics kernel; every CTA waits for it before exiting,
+    // so the GEMM's wait on this grid covers both
+    grid_dep_wait();
+    uint64_t Ap[16], Bp[32];
+    if (KIND == 1) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) Ap[i] = p.Ap[i];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) Bp[i] = p.Bp[i];
+    }
+    float mh = 0.f, ml = 0.f;
+    int cur_tile = -1;
+    if (DEBUG_XT && CENTER) {
+      // one tile per CTA in the debug launch; the rounding remainders of the means sit in
+      // the first element of each output row until this CTA overwrites its rows
+      const int tile = p.tiles - 1 - static_cast<int>(q0 / PP);
+      const int row = tile * 128 + rl;
+      if (row < p.M) { mh = p.mu[row]; ml = p.mulo[static_cast<int64_t>(row) * p.mulo_stride]; }
+      cur_tile = tile;
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * 4 * kGroups) : "memory");
+    }
+    bool ok = true;
+    for (int64_t q = q0 + g; q < q1 && ok; q += kGroups) {
+      const int tile = p.tiles - 1 - static_cast<int>(q / PP);
+      const int pair = static_cast<int>(q % PP);
+      const int row = tile * 128 + rl;
+      if (CENTER && tile != cur_tile) {
+        cur_tile = tile;
+        mh = row < p.M ? p.mu[row] : 0.f;
+        ml = row < p.M ? p.mulo[static_cast<int64_t>(row) * p.mulo_stride] : 0.f;
+      }
+      if (!CENTER && pair == 0 && p.mu_clear != nullptr) p.mu_clear[row] = 0.f;   // row < m_pad
+      uint32_t sbw = 0;
+      const int64_t n0 = 2 * (q - q0);
+      for (int cc = 0; cc < 2; ++cc) {
+        const int64_t n = n0 + cc;
+        const int s = static_cast<int>(n % kStages);
+        ok = __all_sync(0xffffffffu, mbar_wait(&full[s], static_cast<uint32_t>(n / kStages) & 1u, p.err,
+                                               KQ_DEV_ERR_TIMEOUT_FULL));
+        if (!ok) break;
+        const uint8_t* rowp = stage0 + s * kStageBytes + static_cast<uint32_t>(rl) * 128u;
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          const int b = 4 * pair + 2 * cc + h;
+          if (b >= nb) continue;
+          uint64_t v2[16];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const uint4 w = *reinterpret_cast<const uint4*>(
+                rowp + 16u * (static_cast<uint32_t>(4 * h + c) ^ (static_cast<uint32_t>(rl) & 7u)));
+            v2[4 * c + 0] = bf16x2_to_f2(w.x);
+            v2[4 * c + 1] = bf16x2_to_f2(w.y);
+            v2[4 * c + 2] = bf16x2_to_f2(w.z);
+            v2[4 * c + 3] = bf16x2_to_f2(w.w);
+          }
+          if (CENTER) {
+            const uint64_t m2h = f2pack(mh, mh), m2l = f2pack(ml, ml);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v2[i] = fsub2(fsub2(v2[i], m2h), m2l);
+          }
+          if (KIND == 1) kron_apply2(v2, Ap, Bp);
+          if (DEBUG_XT) {
+            if (row < p.M) {
+              float4* o = reinterpret_cast<float4*>(p.xt + static_cast<size_t>(row) * p.K + b * kBlock);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o[i] = make_float4(f2lo(v2[2 * i]), f2hi(v2[2 * i]), f2lo(v2[2 * i + 1]), f2hi(v2[2 * i + 1]));
+            }
+            continue;
+          }
+          const uint32_t sb = mx_scale_byte(amax32_2(v2));
+          uint32_t c4[4];
+          encode_scaled2(v2, mx_inv_scale(sb), c4);
+          if (row < p.M)
+            *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * (p.K / 2) + b * 16) =
+                make_uint4(c4[0], c4[1], c4[2], c4[3]);
+          sbw |= sb << (8 * (2 * cc + h));
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+      }
+      if (!DEBUG_XT && ok) {
+        // scales of blocks 4 pair .. 4 pair + 3 (0 past the last block); the row's padding
+        // block groups are zeroed with its last pair. Rows M .. m_pad - 1 get zero scales.
+        *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, 4 * pair, p.katoms)) = sbw;
+        if (pair == PP - 1)
+          for (int bb = 4 * PP; bb < nb_pad; bb += 4)
+            *reinterpret_cast<uint32_t*>(p.sf + sf_offset(row, bb, p.katoms)) = 0u;
+      }
+    }
+  }
+}
+
+template <int KIND, int CENTER, bool DBG>
+static cudaError_t launch_chunks_t(const ChunkParams& p, bool dependent, int num_sms, cudaStream_t st) {
+  auto fn = k_quantize_chunks<KIND, CENTER, DBG>;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(chunkq::kSmemBytes));
+  if (e != cudaSuccess) return e;
+  const int64_t items = static_cast<int64_t>(p.tiles) * p.pairs;
+  // the debug launch gives each CTA exactly one row tile (see the remainders above)
+  int64_t grid = DBG ? p.tiles : (items < num_sms ? items : num_sms);
+  if (grid < 1) grid = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(chunkq::kThreads);
+  cfg.dynamicSmemBytes = chunkq::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = dependent ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, fn, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_chunks(const ChunkParams& p, int kind, bool center, bool debug_xt,
+                                   bool dependent, int num_sms, cudaStream_t st) {
+#define KQ_CHUNKS(KD, C)                                                               \
+  if (kind == KD && center == (C != 0))                                                \
+    return debug_xt ? launch_chunks_t<KD, C, true>(p, dependent, num_sms, st)          \
+                    : launch_chunks_t<KD, C, false>(p, dependent, num_sms, st);
+  KQ_CHUNKS(0, 0) KQ_CHUNKS(0, 1) KQ_CHUNKS(1, 0) KQ_CHUNKS(1, 1)
+#undef KQ_CHUNKS
+  return cudaErrorInvalidValue;
 }
 
 // ----------------------------------------------------------------------------------
@@ -868,7 +1160,7 @@ cudaError_t launch_encode_f32(const float* V, int M, int K, uint8_t* codes, uint
   return cudaGetLastError();
 }
 
-cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st) {
+cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st, bool dependent) {
   using namespace lowrank;
   auto fn = p.deep ? k_lowrank_u<kStagesDeep> : k_lowrank_u<kStages>;
   const uint32_t smem = smem_bytes(p.deep ? kStagesDeep : kStages);
@@ -888,7 +1180,7 @@ cudaError_t launch_lowrank_u(const LowRankParams& p, cudaStream_t st) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = dependent ? 2 : 1;
   e = cudaLaunchKernelEx(&cfg, fn, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
