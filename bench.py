@@ -530,7 +530,13 @@ def main():
                   "peak_source": peaks["source"] + " copy bandwidth"}
     roof_g["algorithmic_per_launch"] = gemm_flops if roof_g["unit"] == "TFLOP/s" else gemm_bytes
     q_ach = q_bytes / (q_ms * 1e-3) / 1e9
-    qname = "k_quantize_rows+k_lowrank_u" if w.rank else "k_quantize_rows"
+    # Kronecker (or no) transform without the front-end or the codebook: the statistics +
+    # low-rank kernel, then the streaming quantizer; otherwise the row-staged quantizer
+    streaming = w.transform in ("kron", "none") and ln is None and not lut
+    if streaming:
+        qname = "k_lowrank_u+k_quantize_chunks" if (w.rank or w.center) else "k_quantize_chunks"
+    else:
+        qname = "k_quantize_rows+k_lowrank_u" if w.rank else "k_quantize_rows"
     roof_q = {"kernel": qname, "bound": "hbm", "achieved": q_ach, "peak": peaks["hbm_gbs"],
               "unit": "GB/s", "frac": q_ach / peaks["hbm_gbs"],
               "peak_source": peaks["source"] + " copy bandwidth", "algorithmic_per_launch": q_bytes}

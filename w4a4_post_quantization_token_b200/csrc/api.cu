@@ -457,7 +457,19 @@ kq_status run_chunk_path(const kq_layer_desc* d, const void* weights, const void
                  static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, 64, 128,
                  CU_TENSOR_MAP_SWIZZLE_128B))
     return KQ_ERR_CUDA;
-  if (d->t.kind == KQ_T_KRON) kron_pairs(d, cp.Ap, cp.Bp);
+  if (d->t.kind == KQ_T_KRON) {
+    kron_pairs(d, cp.Ap, cp.Bp);
+    for (int k = 0; k < 4; ++k) {
+      double a = 0.0;
+      for (int i = 0; i < 4; ++i) a += d->t.A[4 * i + k];
+      cp.colsumA[k] = static_cast<float>(a);
+    }
+    for (int l = 0; l < 8; ++l) {
+      double b = 0.0;
+      for (int j = 0; j < 8; ++j) b += d->t.B[8 * j + l];
+      cp.colsumB[l] = static_cast<float>(b);
+    }
+  }
   cp.M = M; cp.K = K;
   cp.m_pad = static_cast<int>(AL.m_pad);
   cp.tiles = static_cast<int>(cdiv(M, 128));

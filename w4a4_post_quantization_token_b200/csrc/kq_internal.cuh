@@ -92,6 +92,8 @@ struct ChunkParams {
   CUtensorMap tmap_x;          // X [M, K] bf16, box 64 x 128, 128-byte swizzle
   uint64_t Ap[16];             // Kronecker A as pairs (A[i][k], A[i][k]), index 4 i + k
   uint64_t Bp[32];             // Kronecker B as pairs (B[j][2l], B[j][2l+1]), index 4 j + l
+  float colsumA[4];            // Kronecker: sum_i A[i][k] and sum_j B[j][l] (1^T P = sA (x) sB)
+  float colsumB[8];
   int M, K, m_pad;
   int tiles;                   // cdiv(M, 128)
   int pairs;                   // pieces of 4 blocks per row: cdiv(K, 128)

@@ -82,6 +82,36 @@ __device__ __forceinline__ void kron_apply2(uint64_t (&v2)[16], const uint64_t (
     }
 }
 
+// kron_apply2 whose second stage starts from bias2[4k + lp] instead of 0: adds a constant
+// per output element in the same pass (used to apply a per-token correction -m (1^T P)).
+__device__ __forceinline__ void kron_apply2_bias(uint64_t (&v2)[16], const uint64_t (&Ap)[16],
+                                                 const uint64_t (&Bp)[32], const uint64_t (&bias2)[16]) {
+  uint64_t t2[16];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint64_t acc[4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const float x = (j & 1) ? f2hi(v2[4 * i + j / 2]) : f2lo(v2[4 * i + j / 2]);
+      const uint64_t xx = f2pack(x, x);
+#pragma unroll
+      for (int lp = 0; lp < 4; ++lp)
+        acc[lp] = j == 0 ? fmul2(xx, Bp[lp]) : ffma2(xx, Bp[4 * j + lp], acc[lp]);
+    }
+#pragma unroll
+    for (int lp = 0; lp < 4; ++lp) t2[4 * i + lp] = acc[lp];
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+#pragma unroll
+    for (int lp = 0; lp < 4; ++lp) {
+      uint64_t acc = ffma2(Ap[k], t2[lp], bias2[4 * k + lp]);
+#pragma unroll
+      for (int i = 1; i < 4; ++i) acc = ffma2(Ap[4 * i + k], t2[4 * i + lp], acc);
+      v2[4 * k + lp] = acc;
+    }
+}
+
 // Unnormalised 32-point Walsh-Hadamard transform (Sylvester order) on pairs.
 __device__ __forceinline__ void fwht32_2(uint64_t (&v2)[16]) {
 #pragma unroll
@@ -991,6 +1021,20 @@ __global__ void __launch_bounds__(chunkq::kThreads, 1) k_quantize_chunks(const _
       for (int i = 0; i < 32; ++i) Bp[i] = p.Bp[i];
     }
     float mh = 0.f, ml = 0.f;
+    // Kronecker + centring: x - mu_hi per element, and the remainder mu_lo enters the
+    // transform's second stage as the constant -mu_lo (1^T P)[8k + l] = -mu_lo sA[k] sB[l]
+    uint64_t bias2[16];
+    auto set_bias = [&](float lo) {
+      if (KIND == 1 && CENTER) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+#pragma unroll
+          for (int lp = 0; lp < 4; ++lp)
+            bias2[4 * k + lp] = f2pack(-lo * p.colsumA[k] * p.colsumB[2 * lp],
+                                       -lo * p.colsumA[k] * p.colsumB[2 * lp + 1]);
+      }
+    };
+    set_bias(0.f);
     int cur_tile = -1;
     if (DEBUG_XT && CENTER) {
       // one tile per CTA in the debug launch; the rounding remainders of the means sit in
@@ -998,6 +1042,7 @@ __global__ void __launch_bounds__(chunkq::kThreads, 1) k_quantize_chunks(const _
       const int tile = p.tiles - 1 - static_cast<int>(q0 / PP);
       const int row = tile * 128 + rl;
       if (row < p.M) { mh = p.mu[row]; ml = p.mulo[static_cast<int64_t>(row) * p.mulo_stride]; }
+      set_bias(ml);
       cur_tile = tile;
       asm volatile("bar.sync 1, %0;" ::"n"(32 * 4 * kGroups) : "memory");
     }
@@ -1010,6 +1055,7 @@ __global__ void __launch_bounds__(chunkq::kThreads, 1) k_quantize_chunks(const _
         cur_tile = tile;
         mh = row < p.M ? p.mu[row] : 0.f;
         ml = row < p.M ? p.mulo[static_cast<int64_t>(row) * p.mulo_stride] : 0.f;
+        set_bias(ml);
       }
       if (!CENTER && pair == 0 && p.mu_clear != nullptr) p.mu_clear[row] = 0.f;   // row < m_pad
       uint32_t sbw = 0;
@@ -1035,12 +1081,17 @@ __global__ void __launch_bounds__(chunkq::kThreads, 1) k_quantize_chunks(const _
             v2[4 * c + 2] = bf16x2_to_f2(w.z);
             v2[4 * c + 3] = bf16x2_to_f2(w.w);
           }
-          if (CENTER) {
+          if (CENTER && KIND == 1) {
+            const uint64_t m2h = f2pack(mh, mh);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v2[i] = fsub2(v2[i], m2h);
+          } else if (CENTER) {
             const uint64_t m2h = f2pack(mh, mh), m2l = f2pack(ml, ml);
 #pragma unroll
             for (int i = 0; i < 16; ++i) v2[i] = fsub2(fsub2(v2[i], m2h), m2l);
           }
-          if (KIND == 1) kron_apply2(v2, Ap, Bp);
+          if (KIND == 1 && CENTER) kron_apply2_bias(v2, Ap, Bp, bias2);
+          else if (KIND == 1) kron_apply2(v2, Ap, Bp);
           if (DEBUG_XT) {
             if (row < p.M) {
               float4* o = reinterpret_cast<float4*>(p.xt + static_cast<size_t>(row) * p.K + b * kBlock);
