@@ -131,9 +131,11 @@ def measured_traffic(kernel: str, workload_label: str):
     import hashlib
     try:
         with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
-            rec = json.load(f).get(kernel)
-        if rec is None or rec.get("workload") != workload_label:
+            recs = [r for r in json.load(f).get("records", [])
+                    if r.get("kernel") == kernel and r.get("workload") == workload_label]
+        if not recs:
             return None
+        rec = recs[0]
         h = hashlib.sha256()
         for src in rec["sources"]:
             with open(os.path.join(ROOT, src), "rb") as f:
@@ -141,7 +143,7 @@ def measured_traffic(kernel: str, workload_label: str):
         if h.hexdigest()[:16] != rec["source_sha256_16"]:
             return None
         return {"bytes": int(rec["dram_read_bytes"]) + int(rec["dram_write_bytes"]),
-                "note": rec.get("note", "")}
+                "note": rec.get("note", "") + f" ({rec.get('profile', '')})"}
     except (OSError, ValueError, KeyError):
         return None
 
@@ -210,8 +212,8 @@ class Clocks:
 def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = None, ln=None,
                         lut: bool = False):
     """Time the CPU oracle's online path (LayerNorm front-end when on, centre, transform,
-    encode, fp64 contraction with both branches) on the first rows of the batch for about
-    budget_s seconds."""
+    encode, fp64 contraction with both branches) on the first rows of the batch, in
+    512-token pieces, for about budget_s seconds of work."""
     from oracle import layer as olayer
     X = inp["X"]
     if ln is not None:
@@ -228,13 +230,11 @@ def oracle_tokens_per_s(w, inp, prep, budget_s: float, max_rows: int | None = No
     else:
         linear = olayer.linear
     linear(X[:8], inp["T"], w.center, prep)                   # warm caches
-    t0 = time.perf_counter()
-    linear(X[:32], inp["T"], w.center, prep)
-    per_row = max((time.perf_counter() - t0) / 32, 1e-6)
-    rows = int(min(max_rows or w.M, max(32, budget_s / per_row)))
+    rows = int(max_rows or w.M)
     t0 = time.perf_counter()
     done = 0
-    while done < rows:
+    # 512-token pieces until about budget_s of work has run (or every token is done)
+    while done < rows and time.perf_counter() - t0 < budget_s:
         n = min(512, rows - done)
         linear(X[done:done + n], inp["T"], w.center, prep)
         done += n
@@ -586,7 +586,13 @@ def main():
     if not args.no_comparator:
         comparator = quantize_comparator(kq, torch, args, w, inp, sets, R, dev)
 
-    launches_per_step = 2 + (1 if w.rank else 0)
+    # launches per step: the streaming path (Kronecker or none) runs the statistics kernel
+    # (when the layer centres or has a low-rank branch) and the quantizer, the row-staged
+    # path the quantizer and the low-rank kernel; then the GEMM
+    if streaming:
+        launches_per_step = (2 if (w.rank or w.center) else 1) + 1
+    else:
+        launches_per_step = 2 + (1 if w.rank else 0)
     line = {
         "metric": METRIC, "value": tokens_per_s, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -598,7 +604,9 @@ def main():
                    "l2": f"{R} rotating buffer sets of {set_bytes / 1e6:.0f} MB (> L2)",
                    "graph": graph is not None},
         "phases_ms": {"quantize": q_ms, "gemm": g_ms,
-                      "how": f"phase-isolated CUDA-graph replays over the same buffer sets, "
+                      "how": f"phase-isolated "
+                             f"{'CUDA-graph replays' if gq is not None else 'eager launches'} "
+                             f"over the same buffer sets, "
                              f"each >= {PHASE_MIN_S * 1e3:.0f} ms ({q_reps} and {g_reps} "
                              f"replays of {R} launches)"},
         "quantize_gbs": q_bytes / (q_ms * 1e-3) / 1e9,
