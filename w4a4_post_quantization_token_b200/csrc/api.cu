@@ -555,6 +555,7 @@ kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* 
     }
     lp.lowrank = 1;
     lp.stats = 0;                        // the means come from the quantize kernel
+    lp.reverse = 1;                      // the quantize kernel's last rows are in L2
     lp.mu = d->center ? reinterpret_cast<const float*>(act + AL.mu) : nullptr;
     lp.u = reinterpret_cast<uint16_t*>(act + AL.u);
     lp.M = M; lp.K = d->K; lp.split = u_split(M, d->K);

@@ -77,6 +77,7 @@ struct LowRankParams {
   const float* mu;             // [M] token means (null without centring, unused with stats)
   uint16_t* u;                 // U [M, 64] fp16
   int deep;                    // 1: the quantize CTAs leave no room on the SM, use the deep ring
+  int reverse;                 // 1: take the row tiles from the last to the first (after k_quantize_rows)
   int ln;                      // LayerNorm front-end: L1 map is diag(gamma) L1', and
   const float* cg;             //   U = rstd acc - rstd m cg + cb - mu c1 with cg = gamma^T L1'
   const float* cb;             //   and cb = beta^T L1' [64]

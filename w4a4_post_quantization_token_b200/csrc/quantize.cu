@@ -778,7 +778,12 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
   double* psum = reinterpret_cast<double*>(stage0 + kStages * kStageBytes);   // [128] (S > 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int mt = blockIdx.x, ks = blockIdx.y, S = gridDim.y;
+  // After the row-staged quantizer (`reverse`) the row tiles are taken from the last to the
+  // first: that kernel's band of rows moves from the first row to the last, so the rows
+  // it read last are still in L2 when these CTAs start. As the first kernel of the
+  // streaming path the natural order is kept (the streaming quantizer walks backwards).
+  const int mt = p.reverse ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
+  const int ks = blockIdx.y, S = gridDim.y;
   const int m0 = mt * kTileM;
   const int KT = static_cast<int>(cdiv(p.K, kChunkK));
   const bool lr = p.lowrank != 0, stats = p.stats != 0;
@@ -786,7 +791,7 @@ __global__ void __launch_bounds__(192, 1) k_lowrank_u(const __grid_constant__ Lo
   // that at any time they read neighbouring 128-byte pieces of the same rows
   const int nk = KT > ks ? (KT - ks + S - 1) / S : 0;
   // first kernel of a call: clear the device error word (see k_quantize_rows)
-  if (p.clear_err && mt == 0 && ks == 0 && threadIdx.x == 0 && p.err != nullptr) *p.err = 0u;
+  if (p.clear_err && blockIdx.x == 0 && ks == 0 && threadIdx.x == 0 && p.err != nullptr) *p.err = 0u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
