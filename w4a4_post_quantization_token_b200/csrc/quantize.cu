@@ -1072,7 +1072,9 @@ __global__ void __launch_bounds__(chunkq::kThreads, 1) k_quantize_chunks(const _
                                                KQ_DEV_ERR_TIMEOUT_FULL));
         if (!ok) break;
         const uint8_t* rowp = stage0 + s * kStageBytes + static_cast<uint32_t>(rl) * 128u;
-#pragma unroll 1
+        // both blocks of the piece in one unrolled body: two independent transform chains
+        // for the scheduler (measured 4 % faster on the video-DiT layer than one at a time)
+#pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int b = 4 * pair + 2 * cc + h;
           if (b >= nb) continue;
