@@ -376,13 +376,13 @@ kq_status fill_quant_params(const kq_layer_desc* d, const void* weights, const v
   const int max_warps = d->t.kind == KQ_T_KRON ? kQMaxWarpsKron : kQMaxWarps;
   QuantShape q = choose_quant_shape(K, kSmemMax - p->bufs_off, max_warps);
   if (q.warps == 0) return KQ_ERR_UNSUPPORTED_SHAPE;
-  // With a low-rank branch, prefer a footprint that leaves room for one k_lowrank_u CTA on
-  // the same SM: that kernel is launched as a programmatic dependent and reads the token
-  // means only in its epilogue, so its X stream overlaps this kernel. Exactly 8 warps then:
-  // 256 threads x <= 128 registers plus the low-rank CTA's 192 x ~144 fit the 64 K register
-  // file, and fewer warps would cost this kernel more than the overlap gains. Not for the
-  // Kronecker transform: that kernel is FMA-bound and 16 warps beat the overlap (measured:
-  // video layer 314 -> 295 us).
+  // With a low-rank branch, prefer an 8-warp footprint whose shared memory leaves room for
+  // one k_lowrank_u CTA on the same SM (that kernel is a programmatic dependent and reads
+  // the token means only in its epilogue). The low-rank kernel's 255 registers keep the
+  // two apart all the same (192 x 255 + 256 x 106 exceed the 64 K register file); a
+  // 164-register low-rank epilogue that let them share measured no faster. Not for the
+  // Kronecker transform: that kernel is FMA-bound and 16 warps win (measured: video layer
+  // 314 -> 295 us).
   if (d->rank > 0 && d->t.kind != KQ_T_KRON) {
     const size_t share = kSmemPerSM - 2 * kSmemPerBlockReserved - kLowRankSmemBytes;
     if (p->bufs_off + rstride <= share) {
@@ -559,8 +559,8 @@ kq_status run_quantize(const kq_layer_desc* d, const void* weights, const void* 
     lp.mu = d->center ? reinterpret_cast<const float*>(act + AL.mu) : nullptr;
     lp.u = reinterpret_cast<uint16_t*>(act + AL.u);
     lp.M = M; lp.K = d->K; lp.split = u_split(M, d->K);
-    // a quantize CTA and a 3-stage low-rank CTA share an SM only when the quantize shape
-    // was chosen for it; otherwise the low-rank grid runs on SMs of its own: deep ring
+    // 3-stage ring when the quantize shape left shared memory for a low-rank CTA beside it,
+    // else the deep ring
     lp.deep = qp.smem_bytes + kLowRankSmemBytes + 2 * kSmemPerBlockReserved > kSmemPerSM ? 1 : 0;
     lp.err = reinterpret_cast<uint32_t*>(act + AL.err);
     if (launch_lowrank_u(lp, st) != cudaSuccess) return KQ_ERR_CUDA;
