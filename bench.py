@@ -522,6 +522,8 @@ def main():
         roof_g = {"kernel": gname, "bound": "tensor", "achieved": ach, "peak": tensor_peak,
                   "unit": "TFLOP/s", "frac": ach / tensor_peak,
                   "frac_of_nominal": ach / nominal_peak, "nominal_peak": nominal_peak,
+                  # context: the same rate against the power-capped (sustained) measurement
+                  "frac_of_sustained": ach / (peaks["bf16_sustained"] * (1.0 if lut else FP4_OVER_BF16)),
                   "peak_source": peaks["source"] + (" burst bf16 (fp16 rate)" if lut else
                                                     " burst bf16 x 4 (FP4 rate)")}
     else:
