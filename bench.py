@@ -148,6 +148,26 @@ def measured_traffic(kernel: str, workload_label: str):
         return None
 
 
+def algorithmic_work(M: int, K: int, N: int, rank: int, center: bool, lut: bool = False,
+                     out_bf16: bool = True):
+    """Roofline numerators of one step: the GEMM's flops (the 4-bit product, the rank-r
+    branch and the rank-1 restore), the GEMM's bytes (every operand read once, Y written
+    once) and the quantize phase's bytes (X read once; codes, scales, means and U written
+    once). The low-rank operands are stored 64 wide whatever the rank."""
+    rp = 64 if rank else 0
+    gemm_flops = 2.0 * M * N * K + 2.0 * M * N * rank + (M * N if center else 0)
+    ybytes = M * N * (2 if out_bf16 else 4)
+    if lut:   # fp16 operand and fp16 residual, no block scales
+        gemm_bytes = M * K * 2 + N * K * 2 + M * rp * 2 + N * rp * 2 + N * 4 + \
+            (M * 4 if center else 0) + ybytes
+        q_bytes = M * K * 2 + M * K * 2 + M * 8 + M * rp * 2
+    else:
+        gemm_bytes = M * K / 2 + N * K / 2 + (M + N) * K / 32 + M * rp * 2 + N * rp * 2 + N * 4 + \
+            (M * 4 if center else 0) + ybytes
+        q_bytes = M * K * 2 + M * K / 2 + M * K / 32 + M * 4 + M * rp * 2
+    return gemm_flops, gemm_bytes, q_bytes
+
+
 # nominal dense ratio FP4 : BF16 on B200 (9 : 2.25 PFLOP/s), and the nominal dense peaks
 FP4_OVER_BF16 = 4.0
 NOMINAL_FP4_TFLOPS = 9000.0
@@ -501,17 +521,8 @@ def main():
     # the burst figures: FP4 = 4 x the measured burst bf16 rate (the nominal 9 : 2.25 dense
     # ratio), fp16 = the burst bf16 rate, HBM = the measured copy rate.
     peaks = _peaks()
-    M, K, N, rp = w.M, w.K, w.N, (64 if w.rank else 0)
-    gemm_flops = 2.0 * M * N * K + 2.0 * M * N * w.rank + (M * N if w.center else 0)
-    ybytes = M * N * (2 if out_bf16 else 4)
-    if lut:   # fp16 operand and fp16 residual, no block scales
-        gemm_bytes = M * K * 2 + N * K * 2 + M * rp * 2 + N * rp * 2 + N * 4 + \
-            (M * 4 if w.center else 0) + ybytes
-        q_bytes = M * K * 2 + M * K * 2 + M * 8 + M * rp * 2
-    else:
-        gemm_bytes = M * K / 2 + N * K / 2 + (M + N) * K / 32 + M * rp * 2 + N * rp * 2 + N * 4 + \
-            (M * 4 if w.center else 0) + ybytes
-        q_bytes = M * K * 2 + M * K / 2 + M * K / 32 + M * 4 + M * rp * 2
+    M, K, N = w.M, w.K, w.N
+    gemm_flops, gemm_bytes, q_bytes = algorithmic_work(M, K, N, w.rank, w.center, lut, out_bf16)
     tensor_peak = peaks["bf16"] * (1.0 if lut else FP4_OVER_BF16)
     nominal_peak = NOMINAL_FP16_TFLOPS if lut else NOMINAL_FP4_TFLOPS
     t_tensor = gemm_flops / (tensor_peak * 1e12)

@@ -1,4 +1,5 @@
-"""Host logic of bench.py (CPU): the DRAM-traffic lookup that fills `roofline.traffic`.
+"""Host logic of bench.py (CPU): the DRAM-traffic lookup that fills `roofline.traffic`, and
+the algorithmic work per step that the roofline fractions divide by.
 
 A record applies only to its own (kernel, workload) pair and only while the kernel's
 sources hash to the recorded digest; otherwise the bench reports null rather than a figure
@@ -60,3 +61,29 @@ def test_committed_records_match_tree():
     for r in recs:
         assert _digest(ROOT, r["sources"]) == r["source_sha256_16"], r["kernel"]
         assert r["dram_read_bytes"] > 0 and os.path.exists(os.path.join(ROOT, r["profile"]))
+
+
+def test_algorithmic_work_video_dit():
+    """The roofline numerators of the video-DiT layer (35100 x 3072 -> 3072, centred, r = 64),
+    as the bench lines report them (`algorithmic_per_launch`)."""
+    flops, gbytes, qbytes = bench.algorithmic_work(35100, 3072, 3072, 64, True)
+    assert flops == 676_400_025_600          # 2MNK + 2MNr + MN
+    assert qbytes == 277_570_800             # X + codes + scales + means + U
+    # codes 53.9 MB + residual 4.7 MB + scales 3.7 MB + U 4.5 MB + L2 0.4 MB + s, mu + Y 215.7 MB
+    assert gbytes == 282_989_808
+
+
+def test_algorithmic_work_terms():
+    M, K, N = 256, 1024, 512
+    f0, g0, q0 = bench.algorithmic_work(M, K, N, 0, False)
+    assert f0 == 2 * M * N * K
+    assert q0 == M * K * 2 + M * K / 2 + M * K / 32 + M * 4          # no U without a low-rank branch
+    f1, g1, q1 = bench.algorithmic_work(M, K, N, 5, True)
+    assert f1 - f0 == 2 * M * N * 5 + M * N                          # rank-5 branch + rank-1 restore
+    assert q1 - q0 == M * 64 * 2                                     # U stored 64 wide
+    assert g1 - g0 == (M + N) * 64 * 2 + M * 4                       # U, L2 and the means
+    _, g32, _ = bench.algorithmic_work(M, K, N, 0, False, out_bf16=False)
+    assert g32 - g0 == M * N * 2                                     # fp32 Y instead of bf16
+    _, glut, qlut = bench.algorithmic_work(M, K, N, 0, False, lut=True)
+    assert glut - g0 == (M + N) * K * 2 - (M + N) * K / 2 - (M + N) * K / 32   # fp16 operands, no scales
+    assert qlut == M * K * 2 + M * K * 2 + M * 8                     # fp16 operand out, mean and sigma
